@@ -1,0 +1,145 @@
+/*
+ * fipa.h -- C ABI of the fused Invariant Point Attention forward (B200, sm_100a).
+ *
+ * The operation is the IPA aggregation core defined on the BioTorch problem
+ * page "Invariant point attention (IPA)", section "Required behavior":
+ * frames applied to every query/key/value point, the logit
+ *
+ *   L_ijh = q_ih.k_jh / sqrt(3D) + pair_bias_ijh / sqrt(3)
+ *           - 1/2 softplus(point_w_raw_h) sqrt(2/(27P)) sum_p |T_i q_ihp - T_j k_jhp|^2,
+ *
+ * the mask rule (key j permitted iff mask_i && mask_j && pair_mask_ij), a
+ * stable softmax over j (all-zero row for an empty neighbourhood), the
+ * scalar / pair / global-point aggregation, the inverse frame transform of
+ * the aggregated points, the point-length features, the head-major feature
+ * concatenation and the affine output projection (zero update for an empty
+ * neighbourhood).
+ *
+ * The pair representation is given in the factorised form of "Flash
+ * Invariant Point Attention" (FlashIPA): z_ij[c] = sum_r z1[i,r,c] z2[j,r,c]
+ * with factors of shape (B, L, r, d); the per-head pair logit is its
+ * projection pair_bias_ijh = sum_c z_ij[c] Wb[c,h], and the aggregated pair
+ * value is sum_j a_hij z_ij.  No B x N x N tensor is written to device
+ * memory by the forward (except the optional attention output).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the handle's device, owned
+ *     by the caller, contiguous row-major, 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Entry points return a status; they never abort, throw or trap.  A call
+ *     that fails validation launches nothing.  fipa_last_error() gives a
+ *     one-line reason for the handle's most recent failure.
+ *   - fipa_forward allocates nothing and does not synchronise; its kernels run
+ *     asynchronously on `stream`.  One handle must not be used by two streams
+ *     at the same time (its status word is shared).
+ */
+#ifndef FIPA_H
+#define FIPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FIPA_OK = 0,
+  FIPA_ERR_INVALID_ARG = 1,     /* null / misaligned pointer, non-positive dim, bad enum */
+  FIPA_ERR_UNSUPPORTED = 2,     /* valid request outside what this build implements      */
+  FIPA_ERR_WORKSPACE = 3,       /* workspace pointer NULL or smaller than required        */
+  FIPA_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed (see last_error)     */
+  FIPA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait expired (read by sync_status) */
+  FIPA_ERR_INTERNAL = 6
+} fipa_status;
+
+/* dtype of ALL floating inputs ("all floating tensors are finite with common
+ * dtype", Required behavior).  Outputs are float32 in both modes. */
+typedef enum { FIPA_F32 = 0, FIPA_BF16 = 1 } fipa_dtype;
+
+/* Problem sizes; every field must be > 0 ("All dimensions ... are positive").
+ * F = H * (Dv + 4 Q + Cz) is derived. */
+typedef struct {
+  int B;     /* batch                                  */
+  int N;     /* residues per sample (padded length)    */
+  int H;     /* heads                                  */
+  int D;     /* scalar query/key channels              */
+  int Dv;    /* scalar value channels                  */
+  int P;     /* query/key points per head              */
+  int Q;     /* value points per head                  */
+  int Cz;    /* pair channels (factor width d)         */
+  int R;     /* pair factor rank r                     */
+  int Cout;  /* output channels of w_out               */
+} fipa_dims;
+
+typedef struct fipa_handle fipa_handle;
+
+/* Create a handle on CUDA device `device`.  `max_dims` may be NULL; if given,
+ * later calls with any dim larger than it fail with FIPA_ERR_INVALID_ARG.
+ * Allocates a few bytes of device memory for the status word (the only
+ * allocation the library makes).  *out is NULL on failure. */
+fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims,
+                        fipa_dtype dtype, int device);
+
+/* Bytes of device workspace fipa_forward needs for `dims` (O(B*N), no N^2
+ * term).  Pure host arithmetic; no CUDA call. */
+fipa_status fipa_workspace_size(const fipa_handle* h, const fipa_dims* dims,
+                                size_t* bytes);
+
+/* Fused IPA forward.
+ *   q, k        [B,N,H,D]            scalar queries / keys (projected)
+ *   v           [B,N,H,Dv]           scalar values
+ *   q_pts,k_pts [B,N,H,P,3]          LOCAL query / key points
+ *   v_pts       [B,N,H,Q,3]          LOCAL value points
+ *   rot         [B,N,3,3]            proper rotations, column-vector convention
+ *   trans       [B,N,3]              translations: T_i(x) = rot_i @ x + trans_i
+ *   z1, z2      [B,N,R,Cz]           pair factors, z_ij[c] = sum_r z1[i,r,c] z2[j,r,c]
+ *   Wb          [Cz,H]               per-head projection of the pair representation
+ *   point_w_raw [H]                  raw distance weight (softplus applied inside)
+ *   (all of the above: float32 or bfloat16 as fixed at fipa_create)
+ *   mask        [B,N]   uint8        1 = valid residue
+ *   pair_mask   [B,N,N] uint8 or NULL (NULL = all pairs allowed)
+ *   w_out       [F,Cout], b_out [Cout]  (input dtype)
+ *   eps         > 0, used only inside the output point-length square root
+ * Outputs (float32, written for every row including padded / empty ones):
+ *   out_update        [B,N,Cout]     zero for an empty neighbourhood
+ *   out_local_points  [B,N,H,Q,3]    zero for an empty neighbourhood
+ *   out_attention     [B,H,N,N] or NULL: the normalised attention, recomputed
+ *                     by a separate validation kernel (O(N^2) memory and time)
+ *   out_lse           [B,H,N] or NULL: natural-log logsumexp of the permitted
+ *                     logits of each row, -inf for an empty neighbourhood
+ * workspace: device buffer of >= fipa_workspace_size() bytes, 256-byte aligned,
+ * contents undefined on entry and exit. */
+fipa_status fipa_forward(fipa_handle* h,
+                         const void* q, const void* k, const void* v,
+                         const void* q_pts, const void* k_pts, const void* v_pts,
+                         const void* rot, const void* trans,
+                         const void* z1, const void* z2, const void* Wb,
+                         const void* point_w_raw,
+                         const uint8_t* mask, const uint8_t* pair_mask,
+                         const void* w_out, const void* b_out, double eps,
+                         const fipa_dims* dims,
+                         float* out_update, float* out_local_points,
+                         float* out_attention, float* out_lse,
+                         void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Wait for `stream`, then read and clear the handle's device status word.
+ * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
+ * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */
+fipa_status fipa_sync_status(fipa_handle* h, void* stream);
+
+/* Static description of a status code. */
+const char* fipa_status_string(fipa_status s);
+
+/* One-line reason for the handle's most recent failure ("" if none).
+ * The string is owned by the handle and valid until its next call. */
+const char* fipa_last_error(const fipa_handle* h);
+
+/* Release the handle and its status word.  NULL is accepted. */
+fipa_status fipa_destroy(fipa_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FIPA_H */

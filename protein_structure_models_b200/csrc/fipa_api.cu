@@ -1,0 +1,269 @@
+// fipa_api.cu -- the C ABI of include/fipa.h: validation, planning, TMA
+// descriptors and kernel launches.  No allocation per call, no host sync in
+// fipa_forward, status codes instead of exceptions.
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "fipa.h"
+#include "kernels.h"
+
+#define FIPA_API extern "C" __attribute__((visibility("default")))
+
+using fipa::Plan;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct fipa_handle {
+  int device = 0;
+  fipa_dtype dtype = FIPA_BF16;
+  bool has_max = false;
+  fipa_dims max_dims{};
+  int* d_status = nullptr;
+  unsigned long long timeout_ns = 2000000000ull;
+  EncodeTiledFn encode = nullptr;
+  std::string last_error;
+};
+
+namespace {
+
+struct DeviceGuard {
+  int prev = -1, want;
+  explicit DeviceGuard(int d) : want(d) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    if (prev != want) cudaSetDevice(want);
+  }
+  ~DeviceGuard() {
+    if (prev >= 0 && prev != want) cudaSetDevice(prev);
+  }
+};
+
+fipa_status fail(fipa_handle* h, fipa_status s, const std::string& msg) {
+  if (h != nullptr) h->last_error = msg;
+  return s;
+}
+
+fipa_status cuda_fail(fipa_handle* h, const char* what, cudaError_t e) {
+  return fail(h, FIPA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 16-bit row-major tensor [outer, rows, cols] as a TMA map with a 64 x `box_rows`
+// box and 128-byte swizzle (cols is a multiple of 64, so rows are 128-B aligned).
+fipa_status encode_rows(fipa_handle* h, CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                        uint64_t outer, uint32_t box_rows, cuuint32_t rank, const char* what) {
+  cuuint64_t dims[3] = {cols, rows, outer};
+  cuuint64_t strides[2] = {cols * 2, cols * rows * 2};
+  cuuint32_t box[3] = {64, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(h, FIPA_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (" +
+                                      std::to_string((int)r) + ")");
+  return FIPA_OK;
+}
+
+int plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
+  const char* why = "";
+  int rc = fipa::make_plan(p, d->B, d->N, d->H, d->D, d->Dv, d->P, d->Q, d->Cz, d->R, d->Cout,
+                           h->dtype == FIPA_F32 ? 1 : 0, &why);
+  if (rc != 0) h->last_error = why;
+  return rc;
+}
+
+}  // namespace
+
+FIPA_API const char* fipa_status_string(fipa_status s) {
+  switch (s) {
+    case FIPA_OK: return "ok";
+    case FIPA_ERR_INVALID_ARG: return "invalid argument";
+    case FIPA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FIPA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FIPA_ERR_CUDA: return "CUDA error";
+    case FIPA_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case FIPA_ERR_INTERNAL: return "internal error";
+  }
+  return "unknown status";
+}
+
+FIPA_API const char* fipa_last_error(const fipa_handle* h) {
+  return h == nullptr ? "" : h->last_error.c_str();
+}
+
+FIPA_API fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims, fipa_dtype dtype, int device) {
+  if (out == nullptr) return FIPA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (dtype != FIPA_F32 && dtype != FIPA_BF16) return FIPA_ERR_INVALID_ARG;
+  if (device < 0) return FIPA_ERR_INVALID_ARG;
+  if (max_dims != nullptr) {
+    const int* f = &max_dims->B;
+    for (int k = 0; k < 10; ++k)
+      if (f[k] <= 0) return FIPA_ERR_INVALID_ARG;
+  }
+  int count = 0;
+  if (cudaGetDeviceCount(&count) != cudaSuccess || device >= count) return FIPA_ERR_CUDA;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  if (major != 10 || minor != 0) return FIPA_ERR_UNSUPPORTED;   // built for sm_100a only
+  fipa_handle* h = new (std::nothrow) fipa_handle();
+  if (h == nullptr) return FIPA_ERR_INTERNAL;
+  h->device = device;
+  h->dtype = dtype;
+  if (max_dims != nullptr) { h->has_max = true; h->max_dims = *max_dims; }
+  if (const char* env = std::getenv("FIPA_WAIT_TIMEOUT_MS")) {
+    const long ms = std::strtol(env, nullptr, 10);
+    if (ms > 0) h->timeout_ns = (unsigned long long)ms * 1000000ull;
+  }
+  DeviceGuard g(device);
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    delete h;
+    return FIPA_ERR_CUDA;
+  }
+  h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  if (cudaMalloc(&h->d_status, 256) != cudaSuccess || cudaMemset(h->d_status, 0, 256) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    if (h->d_status) cudaFree(h->d_status);
+    delete h;
+    return FIPA_ERR_CUDA;
+  }
+  *out = h;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_destroy(fipa_handle* h) {
+  if (h == nullptr) return FIPA_OK;
+  {
+    DeviceGuard g(h->device);
+    if (h->d_status) cudaFree(h->d_status);
+  }
+  delete h;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_workspace_size(const fipa_handle* hc, const fipa_dims* dims, size_t* bytes) {
+  fipa_handle* h = const_cast<fipa_handle*>(hc);
+  if (h == nullptr || dims == nullptr || bytes == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "null argument");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  *bytes = p.total;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_sync_status(fipa_handle* h, void* stream) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  DeviceGuard g(h->device);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, "stream", e);
+  int code = 0;
+  e = cudaMemcpy(&code, h->d_status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, "status read", e);
+  if (code != 0) {
+    cudaMemset(h->d_status, 0, sizeof(int));
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "device wait timed out (code %d, site %d)", code & 0xff, code >> 8);
+    return fail(h, FIPA_ERR_DEVICE_TIMEOUT, buf);
+  }
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                  const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                  const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                  const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                  const void* b_out, double eps, const fipa_dims* dims, float* out_update,
+                                  float* out_local_points, float* out_attention, float* out_lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  if (h->has_max) {
+    const int* a = &dims->B;
+    const int* m = &h->max_dims.B;
+    for (int i = 0; i < 10; ++i)
+      if (a[i] > m[i]) return fail(h, FIPA_ERR_INVALID_ARG, "dims exceed the handle's max_dims");
+  }
+  const size_t es = h->dtype == FIPA_F32 ? 4 : 2;
+  const void* req[] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, w_out, b_out};
+  const char* names[] = {"q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "Wb",
+                         "point_w_raw", "w_out", "b_out"};
+  for (int i = 0; i < 14; ++i) {
+    if (req[i] == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is NULL");
+    if (!aligned(req[i], es)) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is misaligned");
+  }
+  if (mask == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "mask is NULL");
+  if (out_update == nullptr || out_local_points == nullptr)
+    return fail(h, FIPA_ERR_INVALID_ARG, "out_update / out_local_points is NULL");
+  if (!aligned(out_update, 4) || !aligned(out_local_points, 4) || !aligned(out_attention, 4) || !aligned(out_lse, 4))
+    return fail(h, FIPA_ERR_INVALID_ARG, "output pointer misaligned");
+  if (!(eps > 0.0) || !std::isfinite(eps)) return fail(h, FIPA_ERR_INVALID_ARG, "eps must be finite and > 0");
+  if (workspace == nullptr || workspace_bytes < p.total)
+    return fail(h, FIPA_ERR_WORKSPACE, "workspace needs " + std::to_string(p.total) + " bytes");
+  if (!aligned(workspace, 256)) return fail(h, FIPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+
+  DeviceGuard g(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  fipa::Work w;
+  w.Q = reinterpret_cast<__half*>(ws + p.off_Q);
+  w.KH = reinterpret_cast<__half*>(ws + p.off_KH);
+  w.VH = reinterpret_cast<__half*>(ws + p.off_VH);
+  w.Z = reinterpret_cast<__half*>(ws + p.off_Z);
+  w.kvec = reinterpret_cast<float4*>(ws + p.off_kvec);
+  w.qvec = reinterpret_cast<float4*>(ws + p.off_qvec);
+  w.orig = reinterpret_cast<float4*>(ws + p.off_orig);
+  w.flag = reinterpret_cast<int*>(ws + p.off_flag);
+  w.O = reinterpret_cast<float*>(ws + p.off_O);
+  w.W = reinterpret_cast<float4*>(ws + p.off_W);
+  w.stats = reinterpret_cast<float2*>(ws + p.off_stats);
+  w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
+  w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
+  w.rowflag = ws + p.off_rowflag;
+
+  fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
+                  w_out, b_out, (float)eps};
+  fipa::Outputs out{out_update, out_local_points, out_attention, out_lse};
+  fipa::DeviceCtl ctl{h->d_status, h->timeout_ns};
+  const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
+
+  CUtensorMap tmQ, tmKH, tmVH, tmZ, tmA, tmB;
+  fipa_status st;
+  if ((st = encode_rows(h, &tmQ, w.Q, p.Kq, N, BH, 128, 3, "Qhat")) != FIPA_OK) return st;
+  if ((st = encode_rows(h, &tmKH, w.KH, p.KHp, N, BH, 128, 3, "Khat")) != FIPA_OK) return st;
+  if ((st = encode_rows(h, &tmVH, w.VH, p.VHp, N, BH, 128, 3, "Vhat")) != FIPA_OK) return st;
+  if ((st = encode_rows(h, &tmZ, w.Z, p.Zp, N, B, 128, 3, "Z")) != FIPA_OK) return st;
+  if ((st = encode_rows(h, &tmA, w.feat, p.Kgp, B * N, 1, 128, 2, "features")) != FIPA_OK) return st;
+  if ((st = encode_rows(h, &tmB, w.wT, p.Kgp, (uint64_t)fipa::rup(p.Cout, p.ntile_out), 1, p.ntile_out, 2,
+                        "w_out")) != FIPA_OK)
+    return st;
+
+  cudaError_t e;
+  if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
+  if ((e = fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s)) != cudaSuccess)
+    return cuda_fail(h, "core launch", e);
+  if ((e = fipa::launch_weight_prep(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "weight prep launch", e);
+  if ((e = fipa::launch_features(p, in, w, out, s)) != cudaSuccess) return cuda_fail(h, "features launch", e);
+  if ((e = fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s)) != cudaSuccess)
+    return cuda_fail(h, "output projection launch", e);
+  if (out_attention != nullptr) {
+    if ((e = fipa::launch_attention_dump(p, in, w, out, s)) != cudaSuccess)
+      return cuda_fail(h, "attention launch", e);
+  }
+  return FIPA_OK;
+}

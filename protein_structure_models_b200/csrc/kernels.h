@@ -1,0 +1,66 @@
+// kernels.h -- argument blocks and launchers of the fused IPA forward kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "plan.h"
+
+namespace fipa {
+
+// Inputs exactly as the C ABI receives them (dtype fixed by Plan::f32).
+struct Inputs {
+  const void *q, *k, *v, *q_pts, *k_pts, *v_pts, *rot, *trans, *z1, *z2, *Wb, *raw;
+  const uint8_t* mask;
+  const uint8_t* pair_mask;   // may be null
+  const void *w_out, *b_out;
+  float eps;
+};
+
+// Workspace views (see plan.h for the layouts).
+struct Work {
+  __half *Q, *KH, *VH, *Z;
+  float4 *kvec;    // [B*H, N] {-g sum_p |b'|^2 (or -inf if masked), sum_p b'}
+  float4 *qvec;    // [B*H, N] {sum_p a', -g sum_p |a'|^2}
+  float4 *orig;    // [B, nT]  {tile origin xyz, valid residues in tile}
+  int *flag;       // [B, nT]  tile has a valid residue
+  float *O;        // [B, N, H, Ocols] normalised aggregates of the lifted value columns
+  float4 *W;       // [B, N, H]  {sum_j a_ij o_T(j) (xyz), l}
+  float2 *stats;   // [B, H, N]  {running max M (log2 units), softmax denominator l}
+  __half *feat;    // [B*N, Kgp] output-projection operand (feature hi/lo halves)
+  __half *wT;      // [Cout_pad, Kgp] output-projection weights, K-major
+  uint8_t *rowflag;// [B*N] row has a non-empty neighbourhood
+};
+
+struct Outputs {
+  float *update, *local_points, *attention, *lse;
+};
+
+struct DeviceCtl {
+  int *status;
+  unsigned long long timeout_ns;
+};
+
+// Launchers return the cudaError_t of the launch.
+cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
+                        const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
+                        const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s);
+cudaError_t launch_features(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
+                            cudaStream_t s);
+cudaError_t launch_weight_prep(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s);
+cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
+                            const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl,
+                            cudaStream_t s);
+cudaError_t launch_attention_dump(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
+                                  cudaStream_t s);
+
+// Per-head distance weight 1/2 softplus(raw) sqrt(2/(27P)), softplus without overflow.
+__device__ __forceinline__ float point_weight(float raw, int P) {
+  const float sp = raw > 0.f ? raw + log1pf(expf(-raw)) : log1pf(expf(raw));
+  return 0.5f * sp * sqrtf(2.0f / (27.0f * (float)P));
+}
+
+}  // namespace fipa

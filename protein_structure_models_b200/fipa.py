@@ -1,0 +1,194 @@
+"""ctypes binding of libfipa.so (include/fipa.h).  Argument marshalling only.
+
+Every step of the forward runs in the CUDA library; this module checks
+shapes/dtypes of torch tensors, allocates outputs and the workspace with torch,
+and passes raw device pointers and the current CUDA stream.  There is no
+fallback: if the library is missing or the call fails, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfipa.so")
+
+FIPA_OK = 0
+STATUS_NAMES = {0: "FIPA_OK", 1: "FIPA_ERR_INVALID_ARG", 2: "FIPA_ERR_UNSUPPORTED",
+                3: "FIPA_ERR_WORKSPACE", 4: "FIPA_ERR_CUDA", 5: "FIPA_ERR_DEVICE_TIMEOUT",
+                6: "FIPA_ERR_INTERNAL"}
+F32, BF16 = 0, 1
+DIM_FIELDS = ("B", "N", "H", "D", "Dv", "P", "Q", "Cz", "R", "Cout")
+
+
+class FipaDims(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_int) for f in DIM_FIELDS]
+
+
+class FipaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libfipa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(f"libfipa.so not found at {_LIB_PATH}; build it with "
+                           "`python -m protein_structure_models_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, c_int, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.fipa_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(FipaDims), c_int, c_int]
+    lib.fipa_create.restype = c_int
+    lib.fipa_workspace_size.argtypes = [vp, ctypes.POINTER(FipaDims), ctypes.POINTER(sz)]
+    lib.fipa_workspace_size.restype = c_int
+    lib.fipa_forward.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double,
+                                                                ctypes.POINTER(FipaDims)] \
+        + [vp] * 4 + [vp, sz, vp]
+    lib.fipa_forward.restype = c_int
+    lib.fipa_sync_status.argtypes = [vp, vp]
+    lib.fipa_sync_status.restype = c_int
+    lib.fipa_status_string.argtypes = [c_int]
+    lib.fipa_status_string.restype = ctypes.c_char_p
+    lib.fipa_last_error.argtypes = [vp]
+    lib.fipa_last_error.restype = ctypes.c_char_p
+    lib.fipa_destroy.argtypes = [vp]
+    lib.fipa_destroy.restype = c_int
+    _lib = lib
+    return lib
+
+
+def make_dims(**kw) -> FipaDims:
+    return FipaDims(*[int(kw[f]) for f in DIM_FIELDS])
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+INPUT_KEYS = ("q", "k", "v", "q_points", "k_points", "v_points", "rotation", "translation",
+              "z1", "z2", "Wb", "point_weight_raw")
+
+
+class Fipa:
+    """One library handle (one device, one input dtype)."""
+
+    def __init__(self, dtype: str = "bf16", device: int = 0, max_dims: Optional[dict] = None):
+        self.lib = load_library()
+        self.dtype = dtype
+        self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        self.device = device
+        h = ctypes.c_void_p()
+        md = make_dims(**max_dims) if max_dims else None
+        st = self.lib.fipa_create(ctypes.byref(h), ctypes.byref(md) if md else None,
+                                  BF16 if dtype == "bf16" else F32, device)
+        if st != FIPA_OK:
+            raise FipaError(st, "fipa_create failed")
+        self.handle = h
+
+    def close(self):
+        if getattr(self, "handle", None):
+            self.lib.fipa_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st):
+        if st != FIPA_OK:
+            raise FipaError(st, self.lib.fipa_last_error(self.handle).decode())
+
+    def workspace_size(self, dims: dict) -> int:
+        d = make_dims(**dims)
+        n = ctypes.c_size_t()
+        self._check(self.lib.fipa_workspace_size(self.handle, ctypes.byref(d), ctypes.byref(n)))
+        return int(n.value)
+
+    def dims_of(self, inp: dict) -> dict:
+        B, N, H, D = inp["q"].shape
+        return dict(B=B, N=N, H=H, D=D, Dv=inp["v"].shape[-1], P=inp["q_points"].shape[3],
+                    Q=inp["v_points"].shape[3], Cz=inp["z1"].shape[3], R=inp["z1"].shape[2],
+                    Cout=inp["w_out"].shape[1])
+
+    def forward(self, inp: dict, eps: float = 1e-8, want_attention: bool = False,
+                want_lse: bool = False, workspace: Optional[torch.Tensor] = None,
+                out: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None) -> dict:
+        """Run fipa_forward on torch tensors (see workloads.make_inputs for keys/layouts)."""
+        dev = torch.device("cuda", self.device)
+        for k in INPUT_KEYS + ("w_out", "b_out"):
+            t = inp[k]
+            if t.dtype != self.torch_dtype or t.device != dev or not t.is_contiguous():
+                raise ValueError(f"{k}: need a contiguous {self.torch_dtype} tensor on {dev}")
+        mask = inp["mask"]
+        pair_mask = inp.get("pair_mask")
+        for name, t in (("mask", mask), ("pair_mask", pair_mask)):
+            if t is not None and (t.dtype not in (torch.bool, torch.uint8) or t.device != dev
+                                  or not t.is_contiguous()):
+                raise ValueError(f"{name}: need a contiguous bool/uint8 tensor on {dev}")
+        dims = self.dims_of(inp)
+        B, N, H, Q, Cout = dims["B"], dims["N"], dims["H"], dims["Q"], dims["Cout"]
+        if out is None:
+            out = {"update": torch.empty((B, N, Cout), dtype=torch.float32, device=dev),
+                   "local_points": torch.empty((B, N, H, Q, 3), dtype=torch.float32, device=dev)}
+            if want_attention:
+                out["attention"] = torch.empty((B, H, N, N), dtype=torch.float32, device=dev)
+            if want_lse:
+                out["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        if workspace is None:
+            workspace = torch.empty(self.workspace_size(dims), dtype=torch.uint8, device=dev)
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        d = make_dims(**dims)
+        st = self.lib.fipa_forward(
+            self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(mask), _ptr(pair_mask),
+            _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d),
+            _ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("attention")),
+            _ptr(out.get("lse")), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+            ctypes.c_void_p(s.cuda_stream))
+        self._check(st)
+        return out
+
+    def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
+        s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))
+        self._check(self.lib.fipa_sync_status(self.handle, ctypes.c_void_p(s.cuda_stream)))
+
+
+_handles: dict = {}
+
+
+def invariant_point_attention(activations: dict, parameters: dict, masks: dict, structure: dict,
+                              eps: float = 1e-8, return_attention: bool = True) -> dict:
+    """The page's function signature, with the pair representation given as factors.
+
+    activations: q, k, v, q_points, k_points, v_points, z1, z2
+    parameters:  point_weight_raw, Wb, w_out, b_out
+    masks:       mask, pair_mask (optional)
+    structure:   rotation, translation
+    Returns {"update", "local_points"} (+ "attention" when return_attention)."""
+    inp = dict(activations)
+    inp.update(parameters)
+    inp.update(structure)
+    inp["mask"] = masks["mask"]
+    inp["pair_mask"] = masks.get("pair_mask")
+    dt = "bf16" if inp["q"].dtype == torch.bfloat16 else "f32"
+    dev = inp["q"].device.index or 0
+    key = (dt, dev)
+    if key not in _handles:
+        _handles[key] = Fipa(dt, dev)
+    h = _handles[key]
+    out = h.forward(inp, eps=eps, want_attention=return_attention)
+    return out
