@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the fused IPA forward (one JSON line on rank 0).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--impl fipa|reference]
+
+A step is one full forward (prologue, fused attention core, features, output
+projection) over one batch of the workload's synthetic inputs, resident in
+HBM.  The L2 cache is flushed (a 256 MB write) between timed steps, outside
+the timed events.  Metric: query-key pairs per second, B*H*N^2 / t (padded
+N), summed over all ranks.  With N > 1 GPUs (torchrun) every rank runs its own
+replica of the workload on its own seed (weak scaling, no collective on the
+data path); the step time is the max over ranks.
+
+--impl reference times the CPU fp64 oracle on the host cores instead (each
+step: one sample of the batch), same metric and unit.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "fused IPA fwd query-key pairs/sec (B·H·N²/s), % of B200 BF16 tensor peak"
+UNIT = "pairs/s"
+DEFAULT_WORKLOAD = "1"
+STAGES_PER_FORWARD = 5          # prologue, core, weight prep, features, output projection
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="0, 1, 2, 4 or 3-<N> (length sweep, N in 512..16384)")
+    ap.add_argument("--impl", choices=("fipa", "reference"), default="fipa")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def dist_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def flops_per_pair(wl) -> int:
+    """Algorithmic lifted-contraction flops per (b,h,i,j): 2 Ka + 2 Va."""
+    ka = wl.D + 3 * wl.P + wl.R * wl.Cz
+    va = wl.Dv + 3 * wl.Q + wl.R * wl.Cz
+    return 2 * ka + 2 * va
+
+
+def pair_counts(wl, inp):
+    valid = inp["mask"].sum(axis=1).astype(np.int64)
+    return wl.B * wl.H * wl.N * wl.N, int(wl.H * np.sum(valid * valid))
+
+
+def workload_config(wl, extra=None):
+    cfg = {"workload": f"{wl.name} ({workloads_key(wl)})", "B": wl.B, "N": wl.N, "H": wl.H, "D": wl.D,
+           "Dv": wl.Dv, "P": wl.P, "Q": wl.Q, "Cz": wl.Cz, "R": wl.R, "Cout": wl.Cout,
+           "input_dtype": wl.dtype, "frames": f"{wl.frames} {wl.t_scale}",
+           "lengths": "all valid" if wl.len_range is None else f"U{{{wl.len_range[0]}..{wl.len_range[1]}}}"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def workloads_key(wl):
+    return f"3-{wl.N}" if wl.index == 3 else str(wl.index)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in out.splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- roofline inputs
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def core_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("core.cu", "sm100.cuh", "plan.h"):
+        with open(os.path.join(ROOT, "protein_structure_models_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(wl):
+    """DRAM bytes per core launch from a committed ncu summary, if it was taken
+    on the current core kernel source for this workload."""
+    path = os.path.join(ROOT, "profiles", f"fipa_core_kernel-{wl.name}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_h = re.search(r"core_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
+    if not m_h or not m_b or m_h.group(1) != core_source_hash():
+        return None
+    return int(m_b.group(1))
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+def cpu_oracle_rate(wl, inp, seconds: float):
+    """Time the fp64 oracle on whole samples of the batch (all query rows) for
+    about `seconds`; returns (pairs/s in B*H*N^2 units, samples, threads, elapsed)."""
+    import oracle
+    done, t0 = 0, time.perf_counter()
+    while True:
+        b = done % wl.B
+        oracle.ipa_forward_dense(workloads.slice_batch(inp, [b]))
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or done >= 4 * wl.B:
+            break
+    return done * wl.H * wl.N * wl.N / el, done, el
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([x.get("num_threads", 1) for x in info] or [1])
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- GPU arm
+def to_device(inp, dtype, dev):
+    import torch
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = {}
+    for k, v in inp.items():
+        if isinstance(v, np.ndarray):
+            t = torch.from_numpy(np.ascontiguousarray(v))
+            out[k] = t.to(dev) if v.dtype == bool else t.to(device=dev, dtype=td)
+        elif v is None:
+            out[k] = None
+    return out
+
+
+def run_fipa(args, wl, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from protein_structure_models_b200 import Fipa
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = workloads.make_inputs(wl, seed=wl.seed + 1000 * rank)
+    d_in = to_device(inp, wl.dtype, dev)
+    h = Fipa(wl.dtype, local_rank)
+    dims = wl.dims()
+    workspace = torch.empty(h.workspace_size(dims), dtype=torch.uint8, device=dev)
+    out = {"update": torch.empty((wl.B, wl.N, wl.Cout), dtype=torch.float32, device=dev),
+           "local_points": torch.empty((wl.B, wl.N, wl.H, wl.Q, 3), dtype=torch.float32, device=dev)}
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)     # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def forward():
+        h.forward(d_in, eps=inp["eps"], workspace=workspace, out=out, stream=stream)
+
+    h.enable_stage_timing(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        forward()
+    torch.cuda.synchronize()
+    h.sync_status()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    stage_sum = {}
+    clocks = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for k in range(args.steps):
+        flush.zero_()                       # outside the timed events
+        ev[k][0].record(stream)
+        forward()
+        ev[k][1].record(stream)
+        for name, ms in h.stage_times().items():   # waits for this step
+            stage_sum[name] = stage_sum.get(name, 0.0) + ms
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    h.sync_status()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    core_ms = stage_sum["core"] / args.steps
+    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms_max = float(t.item())
+
+    # ---- end to end through the public API: pinned host inputs -> device -> result on host
+    host_in = {k: v.cpu().pin_memory() for k, v in d_in.items() if v is not None}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    h.enable_stage_timing(False)
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k, v in host_in.items():
+            d_in[k].copy_(v, non_blocking=True)
+        forward()
+        for k, v in host_out.items():
+            v.copy_(out[k], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_ms = float(t.item())
+    h.sync_status()
+    h.close()
+    return dict(inp=inp, step_ms=step_ms_max, core_ms=core_ms,
+                stage_ms={k: v / args.steps for k, v in stage_sum.items()}, clocks=clk,
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+
+
+def main_fipa(args, wl):
+    rank, world, local_rank = dist_info()
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    r = run_fipa(args, wl, rank, world, local_rank)
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    inp = r["inp"]
+    padded, valid = pair_counts(wl, inp)
+    fpp = flops_per_pair(wl)
+    burst, sustained, hbm, src = measured_peaks()
+    core_s = r["core_ms"] / 1e3
+    achieved = valid * fpp / core_s / 1e12
+    value = padded * world / (r["step_ms"] / 1e3)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, done, el = cpu_oracle_rate(wl, inp, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{done} whole sample(s) of the batch, all query rows, fp64 NumPy, {el:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": workload_config(wl, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                                       "l2": "flushed (256 MB write) between timed steps",
+                                       "math": "fp16 tensor-core products, fp32 accumulate; bf16 inputs"}),
+        "valid_pairs_per_s": valid * world / (r["step_ms"] / 1e3),
+        "stage_ms": r["stage_ms"],
+        "roofline": {"kernel": "fipa_core_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
+                     "peak_source": f"{src} bf16 dense burst (fp16 nominal rate = bf16)",
+                     "work": f"{fpp} flop per valid (b,h,i,j) x {valid} valid pairs per launch",
+                     "traffic": profiled_traffic(wl)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": padded * world / (r["e2e_ms"] / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": STAGES_PER_FORWARD * args.steps,
+        "clocks": r["clocks"],
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- reference arm (oracle)
+def main_reference(args, wl):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return
+    import oracle
+    inp = workloads.make_inputs(wl)
+    sample = [0]
+    for _ in range(args.warmup):
+        oracle.ipa_forward_dense(workloads.slice_batch(inp, sample))
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        oracle.ipa_forward_dense(workloads.slice_batch(inp, [k % wl.B]))
+    el = time.perf_counter() - t0
+    value = args.steps * wl.H * wl.N * wl.N / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": workload_config(wl, {"step": "one sample of the batch, all query rows"}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{args.steps} steps x one sample (B=1 slice), fp64 NumPy oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    wl = workloads.workload(args.workload)
+    if args.impl == "reference":
+        main_reference(args, wl)
+    else:
+        main_fipa(args, wl)
+
+
+if __name__ == "__main__":
+    main()

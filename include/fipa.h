@@ -24,7 +24,8 @@
  *
  * Conventions for every entry point
  *   - All tensor pointers are DEVICE pointers on the handle's device, owned
- *     by the caller, contiguous row-major, 16-byte aligned.
+ *     by the caller, contiguous row-major, aligned to their element size
+ *     (the workspace to 256 bytes).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *   - Entry points return a status; they never abort, throw or trap.  A call
  *     that fails validation launches nothing.  fipa_last_error() gives a
@@ -128,6 +129,19 @@ fipa_status fipa_forward(fipa_handle* h,
  * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */
 fipa_status fipa_sync_status(fipa_handle* h, void* stream);
+
+/* Profiling aid (stage timing).  With `enable` nonzero, later fipa_forward
+ * calls on this handle record a CUDA event before and after each of their
+ * kernels on the call's stream; the events are created here, so fipa_forward
+ * still allocates nothing.  `enable` = 0 turns recording off and frees them. */
+fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable);
+
+/* Device time in milliseconds of each stage of the most recent fipa_forward
+ * recorded with stage timing on, in launch order: [0] prologue, [1] fused
+ * attention core, [2] output-weight preparation, [3] features, [4] output
+ * projection, [5] attention output (0 when not requested).  Waits for that
+ * call's last event.  `n` = capacity of `ms` (up to 6 values are written). */
+fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n);
 
 /* Static description of a status code. */
 const char* fipa_status_string(fipa_status s);

@@ -25,6 +25,8 @@ struct AttnArgs {
   const float4* qvec;
   const float4* orig;
   const float2* stats;
+  const float* QP;
+  const float* KP;
   const uint8_t* mask;
   const uint8_t* pair_mask;
   const void* raw;
@@ -55,25 +57,28 @@ __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
       const float2 st = a.stats[(size_t)bh * N + i];
       M[rr] = st.x; l[rr] = st.y;
       live[rr] = a.mask[(size_t)b * N + i] != 0 && st.y > 0.f;
-      oq[rr] = a.orig[(size_t)b * p.nT + i / kTile];
+      oq[rr] = a.orig[(size_t)b * p.nG + i / kGroup];
       qv[rr] = a.qvec[(size_t)bh * N + i];
     }
   }
   for (int j = threadIdx.x; j < N; j += blockDim.x) {
     const float4 kv = a.kvec[(size_t)bh * N + j];
-    const float4 ok = a.orig[(size_t)b * p.nT + j / kTile];
+    const float4 ok = a.orig[(size_t)b * p.nG + j / kGroup];
     float dot[kRows];
     for (int rr = 0; rr < kRows; ++rr) dot[rr] = 0.f;
     if (kv.x != -INFINITY) {
+      // pair columns first, then the (larger) scalar and point columns, the
+      // accumulation order of the fused core
+      const __half* zrow = a.Z + ((size_t)b * N + j) * p.Zp;
+      for (int c = 0; c < p.Zp; ++c) {
+        const float zc = __half2float(zrow[c]);
+        for (int qz = 0; qz < p.nqz; ++qz)      // every Qhat pair part (u hi, u lo) meets the same z2
+          for (int rr = 0; rr < kRows; ++rr) dot[rr] = fmaf(qs[rr * p.Kq + p.KHp + qz * p.Zp + c], zc, dot[rr]);
+      }
       const __half* krow = a.KH + ((size_t)bh * N + j) * p.KHp;
       for (int c = 0; c < p.KHp; ++c) {
         const float kc = __half2float(krow[c]);
         for (int rr = 0; rr < kRows; ++rr) dot[rr] = fmaf(qs[rr * p.Kq + c], kc, dot[rr]);
-      }
-      const __half* zrow = a.Z + ((size_t)b * N + j) * p.Zp;
-      for (int c = 0; c < p.Zp; ++c) {
-        const float zc = __half2float(zrow[c]);
-        for (int rr = 0; rr < kRows; ++rr) dot[rr] = fmaf(qs[rr * p.Kq + p.KHp + c], zc, dot[rr]);
       }
     }
     for (int rr = 0; rr < kRows; ++rr) {
@@ -85,9 +90,24 @@ __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
       if (permitted) {
         const float dx = oq[rr].x - ok.x, dy = oq[rr].y - ok.y, dz = oq[rr].z - ok.z;
         const float kterm = kv.x + 2.f * g * (dx * kv.y + dy * kv.z + dz * kv.w);
-        const float rc = -g * ((float)p.P * (dx * dx + dy * dy + dz * dz) +
-                               2.f * (dx * qv[rr].x + dy * qv[rr].y + dz * qv[rr].z));
-        const float x = dot[rr] + kterm;
+        float rc, x = dot[rr] + kterm;
+        if (p.geo_simt) {
+          // float32 inputs: exact fp32 squared distance, as in the fused core
+          const int P3 = 3 * p.P;
+          const float* ap = a.QP + ((size_t)bh * N + i) * P3;
+          const float* bp = a.KP + ((size_t)bh * N + j) * P3;
+          float d2 = 0.f;
+          for (int e = 0; e < P3; ++e) {
+            const float dd = (e % 3 == 0) ? dx : (e % 3 == 1) ? dy : dz;
+            const float d = (ap[e] + dd) - bp[e];
+            d2 = fmaf(d, d, d2);
+          }
+          x -= g * d2;
+          rc = 0.f;
+        } else {
+          rc = -g * ((float)p.P * (dx * dx + dy * dy + dz * dz) +
+                     2.f * (dx * qv[rr].x + dy * qv[rr].y + dz * qv[rr].z));
+        }
         att = ex2_approx(fmaf(x, kLog2e, -(M[rr] - rc * kLog2e))) / l[rr];
       }
       a.attention[((size_t)bh * N + i) * N + j] = att;
@@ -99,7 +119,7 @@ __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
 
 cudaError_t launch_attention_dump(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                                   cudaStream_t s) {
-  AttnArgs a{p, w.Q, w.KH, w.Z, w.kvec, w.qvec, w.orig, w.stats, in.mask, in.pair_mask, in.raw,
+  AttnArgs a{p, w.Q, w.KH, w.Z, w.kvec, w.qvec, w.orig, w.stats, w.QP, w.KP, in.mask, in.pair_mask, in.raw,
              out.attention};
   const size_t smem = (size_t)kRows * p.Kq * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(fipa_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

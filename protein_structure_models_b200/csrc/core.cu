@@ -35,6 +35,8 @@ struct CoreArgs {
   Plan p;
   const float4* kvec;
   const float4* qvec;
+  const float* QP;
+  const float* KP;
   const float4* orig;
   const int* flag;
   const uint8_t* mask;
@@ -59,9 +61,11 @@ constexpr int kBarPVDone = 160;
 constexpr int kBarKtFull = 168;    // 2 x u64
 constexpr int kBarKtEmpty = 184;   // 2 x u64
 constexpr int kBarDrain = 200;
-constexpr int kKtBuf = 256;        // 2 x 128 floats
-constexpr int kMisc = 1280;        // tmem slot, abort flag, tile count
-constexpr int kTiles = 2048;       // uint16 key-tile list
+constexpr int kOkBuf = 256;        // 2 x 4 key-group origins (float4)
+constexpr int kMisc = 384;         // tmem slot, abort flag, tile count
+constexpr int kKtBuf = 1024;       // 2 x 4 query groups x 128 keys per-key terms (floats)
+constexpr int kTiles = 5120;       // uint16 key-tile list (<= 1024 entries)
+constexpr int kKpBuf = 7168;       // fp32 key points of two key tiles (float32-input mode)
 
 __device__ __forceinline__ float load_raw(const CoreArgs& a, int h) {
   return a.p.f32 ? static_cast<const float*>(a.raw)[h]
@@ -98,10 +102,12 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* kt_empty = reinterpret_cast<uint64_t*>(tail + kBarKtEmpty);
   uint64_t* drain = reinterpret_cast<uint64_t*>(tail + kBarDrain);
   float* ktbuf = reinterpret_cast<float*>(tail + kKtBuf);
+  float4* okbuf = reinterpret_cast<float4*>(tail + kOkBuf);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + kMisc);
   int* abort_flag = reinterpret_cast<int*>(tail + kMisc + 4);
   int* ntiles = reinterpret_cast<int*>(tail + kMisc + 8);
   uint16_t* tiles = reinterpret_cast<uint16_t*>(tail + kTiles);
+  float* kpbuf = reinterpret_cast<float*>(tail + kKpBuf);          // [2][128][3P] (SPLIT only)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -166,8 +172,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (++st == p.nst) { st = 0; ph ^= 1u; }
       };
       auto push_qk = [&](int kt) {
-        for (int c = 0; c < p.nKH; ++c) push(&tmKH, c * kChunk, kt * kTile, bh);
         for (int c = 0; c < p.nZ; ++c) push(&tmZ, c * kChunk, kt * kTile, b);
+        for (int c = 0; c < p.nKH; ++c) push(&tmKH, c * kChunk, kt * kTile, bh);
       };
       auto push_pv = [&](int kt) {
         for (int c = 0; c < p.nVH; ++c) push(&tmVH, c * kChunk, kt * kTile, bh);
@@ -199,14 +205,24 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const uint32_t idO = idesc_f16(128, 64, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
       auto mma_qk = [&]() -> bool {
-        for (int c = 0; c < p.nQc; ++c) {
+        // key chunks in ring order: the pair part first (each z2 chunk meets nqz
+        // Qhat chunks: u hi, u lo), the head part (scalar and point columns)
+        // last, so the small pair terms accumulate before the large point terms
+        const int nb = p.nZ + p.nKH;
+        for (int c = 0; c < nb; ++c) {
           if (!mbar_wait(&full[st], ph, wc, 3)) return false;
           tc_fence_after();
-          const uint32_t a0 = sQa + c * kChunkBytes, b0 = sRa + st * kChunkBytes;
+          const uint32_t b0 = sRa + st * kChunkBytes;
+          const bool pair = c < p.nZ;
+          const int na = pair ? p.nqz : 1;
+          for (int qz = 0; qz < na; ++qz) {
+            const int ac = pair ? p.nKH + qz * p.nZ + c : c - p.nZ;
+            const uint32_t a0 = sQa + ac * kChunkBytes;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kTmemS, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idS,
-                   (c | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ss(tmem + kTmemS, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idS,
+                     (c | qz | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(&empty[st]);
           if (++st == p.nst) { st = 0; ph ^= 1u; }
         }
@@ -249,37 +265,53 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ per-key terms
-    // kterm_j = -g sum_p |b'_p|^2 + 2g D.sum_p b'_p  (-inf for a masked / absent key)
+    // kterm[s][j] = -g sum_p |b'_p|^2 + 2g D_sj . sum_p b'_p  (-inf for a masked or
+    // absent key), D_sj = origin of query group s - origin of key j's group; the
+    // four key-group origins of the tile go to shared memory as well.
     const int tt = threadIdx.x - 64;
     const float g = point_weight(load_raw(a, h), p.P);
-    const float4 oq = a.orig[(size_t)b * nT + qt];
+    float4 oq[4];
+#pragma unroll
+    for (int sq = 0; sq < 4; ++sq) oq[sq] = a.orig[(size_t)b * p.nG + qt * 4 + sq];
     for (int s = 0; s < nkt; ++s) {
       const int kb = s & 1;
       const bool okw = mbar_wait(&kt_empty[kb], ((s >> 1) & 1) ^ 1, wc, 10);
       if (!__all_sync(0xffffffffu, okw)) break;
       const int kt = tiles[s];
-      const float4 ok4 = a.orig[(size_t)b * nT + kt];
-      const float dx = oq.x - ok4.x, dy = oq.y - ok4.y, dz = oq.z - ok4.z;
+      if (tt < 4) okbuf[kb * 4 + tt] = a.orig[(size_t)b * p.nG + kt * 4 + tt];
       for (int e = tt; e < kTile; e += 64) {
         const int j = kt * kTile + e;
-        float kterm = -INFINITY;
-        if (j < N) {
-          const float4 kv = a.kvec[(size_t)bh * N + j];
-          kterm = kv.x + 2.f * g * (dx * kv.y + dy * kv.z + dz * kv.w);
+        const float4 ok = a.orig[(size_t)b * p.nG + kt * 4 + (e >> 5)];
+        float4 kv = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        if (j < N) kv = a.kvec[(size_t)bh * N + j];
+#pragma unroll
+        for (int sq = 0; sq < 4; ++sq) {
+          const float dx = oq[sq].x - ok.x, dy = oq[sq].y - ok.y, dz = oq[sq].z - ok.z;
+          ktbuf[(kb * 4 + sq) * kTile + e] = SPLIT ? kv.x : kv.x + 2.f * g * (dx * kv.y + dy * kv.z + dz * kv.w);
         }
-        ktbuf[kb * kTile + e] = kterm;
+      }
+      if (SPLIT) {
+        // float32 inputs: the key tile's points b' for the exact fp32 distance
+        const int P3 = 3 * p.P;
+        float* kpb = kpbuf + kb * kTile * P3;
+        const size_t base = ((size_t)bh * N + (size_t)kt * kTile) * P3;
+        const size_t lim = (size_t)(N - kt * kTile) * P3;
+        for (int e = tt; e < kTile * P3; e += 64) kpb[e] = (size_t)e < lim ? a.KP[base + e] : 0.f;
       }
       mbar_arrive(&kt_full[kb]);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
+    // One thread per query row; the warp's TMEM lane quadrant is also the row's
+    // 32-residue origin group.  Per key tile and 32-key group t the row term is
+    // rc_t = -g (P |D_t|^2 + 2 D_t . sum_p a'_p); it rides in the exp's FMA addend.
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const int i = qt * kTile + r;
     const bool in_range = i < N;
     const bool row_valid = in_range && a.mask[(size_t)b * N + i] != 0;
     const float4 qv = in_range ? a.qvec[(size_t)bh * N + i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 oq = a.orig[(size_t)b * nT + qt];
+    const float4 oqs = a.orig[(size_t)b * p.nG + qt * 4 + wq];
     const float g = point_weight(load_raw(a, h), p.P);
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const uint8_t* pmrow = (a.pair_mask != nullptr && in_range) ? a.pair_mask + ((size_t)b * N + i) * N : nullptr;
@@ -288,9 +320,6 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     for (int s = 0; s < nkt; ++s) {
       const int kt = tiles[s];
       const int kb = s & 1;
-      const float4 ok4 = a.orig[(size_t)b * nT + kt];
-      const float dx = oq.x - ok4.x, dy = oq.y - ok4.y, dz = oq.z - ok4.z;
-      const float rc = -g * ((float)p.P * (dx * dx + dy * dy + dz * dz) + 2.f * (dx * qv.x + dy * qv.y + dz * qv.z));
 
       ok = mbar_wait(s_full, s & 1, wc, 7);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
@@ -306,41 +335,71 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
       ok = mbar_wait(&kt_full[kb], (s >> 1) & 1, wc, 11);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      const float4* kb4 = reinterpret_cast<const float4*>(ktbuf + kb * kTile);
-      float mx = -INFINITY;
+      float4 okg[4];
+      float rc[4];
 #pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
+      for (int t = 0; t < 4; ++t) {
+        okg[t] = okbuf[kb * 4 + t];
+        const float dx = oqs.x - okg[t].x, dy = oqs.y - okg[t].y, dz = oqs.z - okg[t].z;
+        rc[t] = SPLIT ? 0.f
+                      : -g * ((float)p.P * (dx * dx + dy * dy + dz * dz) + 2.f * (dx * qv.x + dy * qv.y + dz * qv.z));
+      }
+      const float4* kb4 = reinterpret_cast<const float4*>(ktbuf + (kb * 4 + wq) * kTile);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 kt4 = kb4[(g4 * 32 + e) >> 2];
-          const float x0 = __uint_as_float(sv[g4][e + 0]) + kt4.x;
-          const float x1 = __uint_as_float(sv[g4][e + 1]) + kt4.y;
-          const float x2 = __uint_as_float(sv[g4][e + 2]) + kt4.z;
-          const float x3 = __uint_as_float(sv[g4][e + 3]) + kt4.w;
-          sv[g4][e + 0] = __float_as_uint(x0);
-          sv[g4][e + 1] = __float_as_uint(x1);
-          sv[g4][e + 2] = __float_as_uint(x2);
-          sv[g4][e + 3] = __float_as_uint(x3);
-          mx = fmaxf(mx, fmaxf(fmaxf(x0, x1), fmaxf(x2, x3)));
+          const float4 kt4 = kb4[(t * 32 + e) >> 2];
+          sv[t][e + 0] = __float_as_uint(__uint_as_float(sv[t][e + 0]) + kt4.x);
+          sv[t][e + 1] = __float_as_uint(__uint_as_float(sv[t][e + 1]) + kt4.y);
+          sv[t][e + 2] = __float_as_uint(__uint_as_float(sv[t][e + 2]) + kt4.z);
+          sv[t][e + 3] = __float_as_uint(__uint_as_float(sv[t][e + 3]) + kt4.w);
+        }
+      }
+      if (SPLIT) {
+        // float32 inputs: -g sum_p |a'_p + D_t - b'_p|^2 taken directly in fp32
+        const int P3 = 3 * p.P;
+        const float* kpb = kpbuf + kb * kTile * P3;
+        float aq[3 * kMaxPSimt];
+        for (int x = 0; x < P3; ++x) aq[x] = in_range ? a.QP[((size_t)bh * N + i) * P3 + x] : 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float dd[3] = {oqs.x - okg[t].x, oqs.y - okg[t].y, oqs.z - okg[t].z};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float* kj = kpb + (t * 32 + e) * P3;
+            float d2 = 0.f;
+            for (int x = 0; x < P3; ++x) {
+              const float d = (aq[x] + dd[x % 3]) - kj[x];
+              d2 = fmaf(d, d, d2);
+            }
+            sv[t][e] = __float_as_uint(__uint_as_float(sv[t][e]) - g * d2);
+          }
         }
       }
       mbar_arrive(&kt_empty[kb]);
       if (pmrow != nullptr) {
-        mx = -INFINITY;
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
+        for (int t = 0; t < 4; ++t) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int j = kt * kTile + g4 * 32 + e;
-            if (j >= N || pmrow[j] == 0) sv[g4][e] = __float_as_uint(-INFINITY);
-            mx = fmaxf(mx, __uint_as_float(sv[g4][e]));
+            const int j = kt * kTile + t * 32 + e;
+            if (j >= N || pmrow[j] == 0) sv[t][e] = __float_as_uint(-INFINITY);
           }
         }
       }
-      if (!row_valid) mx = -INFINITY;
+      // tile maximum of the true logits (log2 units, minus -g sum|a'|^2)
+      float mtile = -INFINITY;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sv[t][e]));
+        mtile = fmaxf(mtile, (mx + rc[t]) * kLog2e);
+      }
+      if (!row_valid) mtile = -INFINITY;
 
-      // lazily updated running max (log2 units, true logit minus -g sum|a'|^2)
-      const float mtile = (mx + rc) * kLog2e;
+      // lazily updated running max: rescale only when it grows by more than 2^kTau
       float alpha = 1.f;
       bool resc = false;
       if (mtile > M + kTau) {
@@ -349,34 +408,35 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         M = mtile;
         l *= alpha; Wx *= alpha; Wy *= alpha; Wz *= alpha;
       }
-      const float mb = row_valid ? (M == -INFINITY ? 0.f : M - rc * kLog2e) : INFINITY;
 
       uint32_t pk[2][32];
       uint32_t plo[2][32];
-      float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
 #pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
+      for (int t = 0; t < 4; ++t) {
+        const float mb = row_valid ? (M == -INFINITY ? 0.f : M - rc[t] * kLog2e) : INFINITY;
+        float rs0 = 0.f, rs1 = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[g4][e + 0]), kLog2e, -mb));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[g4][e + 1]), kLog2e, -mb));
-          const float p2 = ex2_approx(fmaf(__uint_as_float(sv[g4][e + 2]), kLog2e, -mb));
-          const float p3 = ex2_approx(fmaf(__uint_as_float(sv[g4][e + 3]), kLog2e, -mb));
-          rs0 += p0; rs1 += p1; rs2 += p2; rs3 += p3;
-          const int w = (g4 & 1) * 16 + e / 2;
-          pk[g4 >> 1][w] = pack_half2(p0, p1);
-          pk[g4 >> 1][w + 1] = pack_half2(p2, p3);
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 0]), kLog2e, -mb));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 1]), kLog2e, -mb));
+          const float p2 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 2]), kLog2e, -mb));
+          const float p3 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 3]), kLog2e, -mb));
+          rs0 += p0 + p1;
+          rs1 += p2 + p3;
+          const int w = (t & 1) * 16 + e / 2;
+          pk[t >> 1][w] = pack_half2(p0, p1);
+          pk[t >> 1][w + 1] = pack_half2(p2, p3);
           if (SPLIT) {
-            const __half2 h01 = *reinterpret_cast<const __half2*>(&pk[g4 >> 1][w]);
-            const __half2 h23 = *reinterpret_cast<const __half2*>(&pk[g4 >> 1][w + 1]);
-            plo[g4 >> 1][w] = pack_half2(p0 - __low2float(h01), p1 - __high2float(h01));
-            plo[g4 >> 1][w + 1] = pack_half2(p2 - __low2float(h23), p3 - __high2float(h23));
+            const __half2 h01 = *reinterpret_cast<const __half2*>(&pk[t >> 1][w]);
+            const __half2 h23 = *reinterpret_cast<const __half2*>(&pk[t >> 1][w + 1]);
+            plo[t >> 1][w] = pack_half2(p0 - __low2float(h01), p1 - __high2float(h01));
+            plo[t >> 1][w + 1] = pack_half2(p2 - __low2float(h23), p3 - __high2float(h23));
           }
         }
+        const float rs = rs0 + rs1;
+        l += rs;
+        Wx += okg[t].x * rs; Wy += okg[t].y * rs; Wz += okg[t].z * rs;
       }
-      const float rs = (rs0 + rs1) + (rs2 + rs3);
-      l += rs;
-      Wx += ok4.x * rs; Wy += ok4.y * rs; Wz += ok4.z * rs;
 
       // P and O are free once the previous P.V product has finished
       if (s > 0) {
@@ -450,7 +510,7 @@ cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Ou
                         const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s) {
   CoreArgs a;
   a.p = p;
-  a.kvec = w.kvec; a.qvec = w.qvec; a.orig = w.orig; a.flag = w.flag;
+  a.kvec = w.kvec; a.qvec = w.qvec; a.QP = w.QP; a.KP = w.KP; a.orig = w.orig; a.flag = w.flag;
   a.mask = in.mask; a.pair_mask = in.pair_mask; a.raw = in.raw;
   a.O = w.O; a.W = w.W; a.stats = w.stats; a.lse = out.lse;
   a.status = ctl.status; a.timeout_ns = ctl.timeout_ns;

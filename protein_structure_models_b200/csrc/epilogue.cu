@@ -63,21 +63,21 @@ __global__ void __launch_bounds__(kFeatWarps * 32) fipa_features_kernel(const Fe
   for (int e = 0; e < 9; ++e) R[e] = ld_in(rot, bi * 9 + e);
 #pragma unroll
   for (int e = 0; e < 3; ++e) t[e] = ld_in(tr, bi * 3 + e);
-  const int gofs = p.nsv * Dv;
+  const int gofs = p.nsv * p.Dv8;
   for (int h = 0; h < H; ++h) {
     const float* orow = a.O + (bi * H + h) * p.Ocols;
     const float4 Wv = a.W[bi * H + h];
     // scalar block
     for (int d = lane; d < Dv; d += 32) {
       float s = orow[d];
-      if (p.f32) s += orow[Dv + d];
+      if (p.f32) s += orow[p.Dv8 + d];
       put_feature(frow, F, p.f32, h * Dv + d, s);
     }
     // points: aggregate in global frame, back into the query frame
     for (int qq = lane; qq < Q; qq += 32) {
       float G[3];
 #pragma unroll
-      for (int x = 0; x < 3; ++x) G[x] = orow[gofs + 3 * qq + x] + orow[gofs + 3 * Q + 3 * qq + x];
+      for (int x = 0; x < 3; ++x) G[x] = orow[gofs + 3 * qq + x] + orow[gofs + p.Q38 + 3 * qq + x];
       G[0] += Wv.x - t[0];
       G[1] += Wv.y - t[1];
       G[2] += Wv.z - t[2];
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kFeatWarps * 32) fipa_features_kernel(const Fe
       float acc = 0.f;
       for (int r = 0; r < p.R; ++r) {
         float u = orow[p.VHp + r * Cz + c];
-        if (p.f32) u += orow[p.VHp + RCz + r * Cz + c];
+        if (p.f32) u += orow[p.VHp + p.RC8 + r * Cz + c];
         acc = fmaf(ld_in(z1, bi * RCz + r * Cz + c), u, acc);
       }
       put_feature(frow, F, p.f32, H * Dv + 4 * H * Q + h * Cz + c, acc);

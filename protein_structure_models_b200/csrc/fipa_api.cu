@@ -27,6 +27,9 @@ struct fipa_handle {
   unsigned long long timeout_ns = 2000000000ull;
   EncodeTiledFn encode = nullptr;
   std::string last_error;
+  bool timing = false;
+  bool timed_call = false;
+  cudaEvent_t ev[7] = {};
 };
 
 namespace {
@@ -141,11 +144,45 @@ FIPA_API fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims, f
   return FIPA_OK;
 }
 
+FIPA_API fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  DeviceGuard g(h->device);
+  if (enable && !h->timing) {
+    for (auto& e : h->ev) {
+      cudaError_t err = cudaEventCreate(&e);
+      if (err != cudaSuccess) return cuda_fail(h, "event create", err);
+    }
+    h->timing = true;
+  } else if (!enable && h->timing) {
+    for (auto& e : h->ev) { cudaEventDestroy(e); e = nullptr; }
+    h->timing = false;
+  }
+  h->timed_call = false;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n) {
+  if (h == nullptr || ms == nullptr || n < 0) return FIPA_ERR_INVALID_ARG;
+  if (!h->timing || !h->timed_call) return fail(h, FIPA_ERR_INVALID_ARG, "no timed fipa_forward call");
+  DeviceGuard g(h->device);
+  cudaError_t e = cudaEventSynchronize(h->ev[6]);
+  if (e != cudaSuccess) return cuda_fail(h, "event sync", e);
+  for (int k = 0; k < 6 && k < n; ++k) {
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, h->ev[k], h->ev[k + 1]);
+    if (e != cudaSuccess) return cuda_fail(h, "event time", e);
+    ms[k] = t;
+  }
+  return FIPA_OK;
+}
+
 FIPA_API fipa_status fipa_destroy(fipa_handle* h) {
   if (h == nullptr) return FIPA_OK;
   {
     DeviceGuard g(h->device);
     if (h->d_status) cudaFree(h->d_status);
+    if (h->timing)
+      for (auto& e : h->ev) cudaEventDestroy(e);
   }
   delete h;
   return FIPA_OK;
@@ -225,6 +262,8 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   w.KH = reinterpret_cast<__half*>(ws + p.off_KH);
   w.VH = reinterpret_cast<__half*>(ws + p.off_VH);
   w.Z = reinterpret_cast<__half*>(ws + p.off_Z);
+  w.QP = reinterpret_cast<float*>(ws + p.off_QP);
+  w.KP = reinterpret_cast<float*>(ws + p.off_KP);
   w.kvec = reinterpret_cast<float4*>(ws + p.off_kvec);
   w.qvec = reinterpret_cast<float4*>(ws + p.off_qvec);
   w.orig = reinterpret_cast<float4*>(ws + p.off_orig);
@@ -254,16 +293,28 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
     return st;
 
   cudaError_t e;
+  const bool rec = h->timing;
+  auto mark = [&](int k) {
+    if (rec) cudaEventRecord(h->ev[k], s);
+  };
+  mark(0);
   if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
+  mark(1);
   if ((e = fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s)) != cudaSuccess)
     return cuda_fail(h, "core launch", e);
+  mark(2);
   if ((e = fipa::launch_weight_prep(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "weight prep launch", e);
+  mark(3);
   if ((e = fipa::launch_features(p, in, w, out, s)) != cudaSuccess) return cuda_fail(h, "features launch", e);
+  mark(4);
   if ((e = fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s)) != cudaSuccess)
     return cuda_fail(h, "output projection launch", e);
+  mark(5);
   if (out_attention != nullptr) {
     if ((e = fipa::launch_attention_dump(p, in, w, out, s)) != cudaSuccess)
       return cuda_fail(h, "attention launch", e);
   }
+  mark(6);
+  h->timed_call = rec;
   return FIPA_OK;
 }

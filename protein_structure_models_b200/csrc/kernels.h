@@ -22,12 +22,13 @@ struct Inputs {
 // Workspace views (see plan.h for the layouts).
 struct Work {
   __half *Q, *KH, *VH, *Z;
+  float *QP, *KP;  // [B*H, N, 3P] a' and b' in fp32 (float32-input mode only)
   float4 *kvec;    // [B*H, N] {-g sum_p |b'|^2 (or -inf if masked), sum_p b'}
   float4 *qvec;    // [B*H, N] {sum_p a', -g sum_p |a'|^2}
-  float4 *orig;    // [B, nT]  {tile origin xyz, valid residues in tile}
+  float4 *orig;    // [B, nG]  {32-residue group origin xyz, valid residues in group}
   int *flag;       // [B, nT]  tile has a valid residue
   float *O;        // [B, N, H, Ocols] normalised aggregates of the lifted value columns
-  float4 *W;       // [B, N, H]  {sum_j a_ij o_T(j) (xyz), l}
+  float4 *W;       // [B, N, H]  {sum_j a_ij o_G(j) (xyz), l}
   float2 *stats;   // [B, H, N]  {running max M (log2 units), softmax denominator l}
   __half *feat;    // [B*N, Kgp] output-projection operand (feature hi/lo halves)
   __half *wT;      // [Cout_pad, Kgp] output-projection weights, K-major

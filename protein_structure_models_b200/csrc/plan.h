@@ -3,24 +3,25 @@
 // Lifted operand layout (FlashIPA, "Flash Invariant Point Attention": the
 // squared-norm expansion |a-b|^2 = |a|^2 - 2 a.b + |b|^2 turns the point
 // term into a dot product; the pair factors z1, z2 turn the pair bias and the
-// pair aggregation into dot products).  Rows are fp16; a 16-bit value that
-// needs more precision is stored as hi + lo halves and the partner operand
-// repeats its own hi half, so hi*hi + hi*lo + lo*hi restores ~22 bits.
+// pair aggregation into dot products).  Rows are fp16; a value that needs
+// more than 11 significant bits is stored as hi + lo halves.
 //
-//   Qhat [B*H, N, Kq]  = [ QH (KHp cols) | QZ (Zp cols) ]
-//       QH   bf16 mode: [ q/sqrt(3D) | 2g a' hi | 2g a' hi | 2g a' lo | 0.. ]
-//            f32  mode: [ q/sqrt(3D) hi | hi | lo | 2g a' hi | hi | lo | 0.. ]
-//       QZ   bf16 mode: [ z1[r,c] Wb[c,h] / sqrt(3) ]          (r-major, then c)
-//            f32  mode: [ u hi | u hi | u lo ]
-//   KH   [B*H, N, KHp]  bf16: [ k | b' hi | b' lo | b' hi | 0.. ]
-//                        f32: [ k hi | lo | hi | b' hi | lo | hi | 0.. ]
-//   Z    [B,   N, Zp ]  bf16: [ z2 ]            f32: [ z2 hi | z2 lo | z2 hi ]
-//   VH   [B*H, N, VHp]  bf16: [ v | g' hi | g' lo | 0.. ]
-//                        f32: [ v hi | v lo | g' hi | g' lo | 0.. ]
-// where a' = T_i(q_p) - o_T, b' = T_j(k_p) - o_T, g' = T_j(v_q) - o_T are
-// global points relative to the mean translation o_T of their own 128-residue
-// tile, and g = the per-head distance weight.  The value side uses the first
-// ZV columns of Z (f32 mode: z2 hi | z2 lo).
+// bfloat16 inputs (the point term runs on the tensor cores):
+//   Qhat [B*H, N, Kq] = [ QH (KHp) | u hi (Zp) | u lo (Zp) ]
+//       QH = [ q/sqrt(3D) | 2g a' hi | 2g a' hi | 2g a' lo | 0.. ],  u = z1[r,c] Wb[c,h]/sqrt(3)
+//   KH   [B*H, N, KHp] = [ k | b' hi | b' lo | b' hi | 0.. ]
+//   Z    [B,   N, Zp ] = [ z2 ]          (exact in fp16; multiplies both u halves)
+//   VH   [B*H, N, VHp] = [ v | g' hi | g' lo | 0.. ]
+// float32 inputs (every value split, the point term in fp32 on the CUDA cores):
+//   QH = [ q/sqrt(3D) hi | hi | lo | 0.. ],  KH = [ k hi | lo | hi | 0.. ]
+//   Qhat pair part = [ u hi | u hi | u lo ],  Z = [ z2 hi | z2 lo | z2 hi ]
+//   VH = [ v hi | v lo | g' hi | g' lo | 0.. ]
+//   QP, KP [B*H, N, 3P] fp32: a' and b' for the exact squared distance
+// where a' = T_i(q_p) - o_G, b' = T_j(k_p) - o_G, g' = T_j(v_q) - o_G are
+// global points relative to the mean translation o_G of the residue's own
+// 32-residue group, and g is the per-head distance weight.  Every column
+// segment is padded to a multiple of 8 columns.  The value product uses the
+// first ZV columns of Z (f32: z2 hi | z2 lo).
 #pragma once
 
 #include <stddef.h>
@@ -29,13 +30,15 @@
 namespace fipa {
 
 constexpr int kTile = 128;       // residues per query / key tile (MMA M and N)
+constexpr int kGroup = 32;       // residues sharing one coordinate origin (4 groups per tile)
 constexpr int kChunk = 64;       // fp16 columns per 128-byte swizzled chunk
 constexpr int kTmemS = 0;        // TMEM column of the logit tile S (128 fp32 columns)
 constexpr int kTmemP = 128;      // TMEM column of P (fp16 pairs: 64 columns, 128 when split)
-constexpr int kMaxQChunks = 8;   // resident Qhat tile <= 128 KB of shared memory
+constexpr int kMaxQChunks = 10;  // resident Qhat tile <= 160 KB of shared memory
 constexpr int kMaxPts = 64;      // points per head handled by the prologue scratch
 constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
-constexpr int kMaxTiles = 2048;  // key tiles per sample (N <= 262144)
+constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
+constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
 
 static inline int cdiv(int a, int b) { return (a + b - 1) / b; }
 static inline int rup(int a, int b) { return cdiv(a, b) * b; }
@@ -45,12 +48,16 @@ struct Plan {
   int B, N, H, D, Dv, P, Q, Cz, R, Cout, F;
   int f32;            // 1: float32 inputs (hi/lo splits everywhere); 0: bfloat16 inputs
   int nT;             // tiles per sample
+  int nG;             // 32-residue origin groups per sample (4 per tile)
   int nsq;            // copies of the scalar q/k columns (1 or 3)
   int nsv;            // copies of the scalar v columns (1 or 2)
   int nz;             // copies of the pair columns on the key side (1 or 3)
   int nzv;            // copies of the pair columns on the value side (1 or 2)
   int KHc, KHp, nKH;  // key/query head-part columns, padded, chunks
   int Zc, Zp, nZ;     // pair columns, padded, chunks
+  int nqz;            // Qhat chunks multiplying each Z chunk (2: u hi and u lo)
+  int D8, P38, Dv8, Q38, RC8;  // segment widths, each padded to 8 columns (one 16-byte chunk)
+  int geo_simt;       // 1: squared distance in fp32 on the CUDA cores (f32 inputs)
   int Kq, nQc;        // Qhat row width and chunks
   int VHc, VHp, nVH;  // value head-part columns, padded, chunks
   int ZVc, nZV;       // pair columns used by the value product, chunks
@@ -59,12 +66,14 @@ struct Plan {
   int tmemO;          // TMEM column of the O accumulator
   int nst;            // shared-memory ring stages of the core kernel
   size_t core_smem;   // dynamic shared memory of the core kernel
+  size_t lift_smem;   // dynamic shared memory of the prologue lift kernel
   int Kg, Kgp;        // output-projection K (2F or 3F) and padded
   int ntile_out;      // output-projection N tile (<= 256)
   int gemm_nst;
   size_t gemm_smem;
   // workspace byte offsets
   size_t off_Q, off_KH, off_VH, off_Z, off_kvec, off_qvec, off_orig, off_flag;
+  size_t off_QP, off_KP;
   size_t off_O, off_W, off_stats, off_feat, off_wT, off_rowflag, total;
 };
 
@@ -81,33 +90,44 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.F = H * (Dv + 4 * Q + Cz);
   p.f32 = f32 ? 1 : 0;
   p.nT = cdiv(N, kTile);
+  p.nG = 4 * p.nT;
   p.nsq = f32 ? 3 : 1;
   p.nsv = f32 ? 2 : 1;
   p.nz = f32 ? 3 : 1;
   p.nzv = f32 ? 2 : 1;
-  p.KHc = p.nsq * D + 9 * P;
+  p.nqz = f32 ? 1 : 2;
+  p.geo_simt = f32 ? 1 : 0;
+  p.D8 = rup(D, 8);
+  p.P38 = rup(3 * P, 8);
+  p.Dv8 = rup(Dv, 8);
+  p.Q38 = rup(3 * Q, 8);
+  p.RC8 = rup(R * Cz, 8);
+  p.KHc = p.nsq * p.D8 + (p.geo_simt ? 0 : 3 * p.P38);
   p.KHp = rup(p.KHc, kChunk);
   p.nKH = p.KHp / kChunk;
-  p.Zc = p.nz * R * Cz;
+  p.Zc = p.nz * p.RC8;
   p.Zp = rup(p.Zc, kChunk);
   p.nZ = p.Zp / kChunk;
-  p.Kq = p.KHp + p.Zp;
+  p.Kq = p.KHp + p.nqz * p.Zp;
   p.nQc = p.Kq / kChunk;
-  p.VHc = p.nsv * Dv + 6 * Q;
+  p.VHc = p.nsv * p.Dv8 + 2 * p.Q38;
   p.VHp = rup(p.VHc, kChunk);
   p.nVH = p.VHp / kChunk;
-  p.ZVc = p.nzv * R * Cz;
+  p.ZVc = p.nzv * p.RC8;
   p.nZV = cdiv(p.ZVc, kChunk);
   p.Ocols = p.VHp + p.nZV * kChunk;
   p.Pcols = f32 ? 128 : 64;
   p.tmemO = kTmemP + p.Pcols;
-  if (p.nT > kMaxTiles) { *why = "N above 262144 is not supported"; return 2; }
+  if (p.nT > kMaxTiles) { *why = "N above 131072 is not supported"; return 2; }
+  if (p.geo_simt && P > kMaxPSimt) { *why = "more than 16 points per head with float32 inputs is not supported"; return 2; }
   if (P > kMaxPts || Q > kMaxPts) { *why = "more than 64 points per head is not supported"; return 2; }
+  if (H > 64) { *why = "more than 64 heads is not supported"; return 2; }
   if (R * Cz > kMaxRCz) { *why = "R*Cz above 1024 is not supported"; return 2; }
-  if (p.nQc > kMaxQChunks) { *why = "lifted query width above 512 columns is not supported"; return 2; }
+  if (p.nQc > kMaxQChunks) { *why = "lifted query width above 640 columns is not supported"; return 2; }
   if (p.tmemO + p.Ocols > 512) { *why = "lifted value width exceeds the 512 tensor-memory columns"; return 2; }
   // core shared memory: resident Qhat + ring + barriers/buffers (+1 KB alignment slack)
-  const size_t fixed = 1024 + 4096 + 2 * kMaxTiles;
+  const size_t kp_bytes = p.geo_simt ? (size_t)2 * kTile * 3 * P * 4 : 0;
+  const size_t fixed = 1024 + 5120 + 2 * kMaxTiles + kp_bytes;   // slack + tail (see core.cu)
   const size_t limit = 232448;  // 227 KB opt-in maximum per block on sm_100
   size_t avail = limit - fixed - (size_t)p.nQc * 16384;
   int nst = (int)(avail / 16384);
@@ -116,6 +136,10 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.nst = nst;
   p.core_smem = fixed + (size_t)(p.nQc + nst) * 16384;
   if (p.core_smem < 120 * 1024) p.core_smem = 120 * 1024;   // one CTA per SM (TMEM is taken whole)
+  // prologue lift kernel: Wb^T, z1 rows, global points, frames of 8 residues
+  p.lift_smem = ((size_t)H * Cz + (size_t)8 * 2 * R * Cz + (size_t)8 * H * (2 * P + Q) * 3 + 8 * 12 +
+                 (size_t)8 * H * (2 * D + Dv)) * 4;
+  if (p.lift_smem > 160 * 1024) { *why = "prologue staging exceeds shared memory (H*Cz or R*Cz too large)"; return 2; }
   // output projection
   p.Kg = (f32 ? 3 : 2) * p.F;
   p.Kgp = rup(p.Kg, kChunk);
@@ -134,9 +158,11 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.off_KH = take(BHN * p.KHp * 2);
   p.off_VH = take(BHN * p.VHp * 2);
   p.off_Z = take(BN * p.Zp * 2);
+  p.off_QP = take(p.geo_simt ? BHN * 3 * P * 4 : 0);
+  p.off_KP = take(p.geo_simt ? BHN * 3 * P * 4 : 0);
   p.off_kvec = take(BHN * 16);
   p.off_qvec = take(BHN * 16);
-  p.off_orig = take((size_t)B * p.nT * 16);
+  p.off_orig = take((size_t)B * p.nG * 16);
   p.off_flag = take((size_t)B * p.nT * 4);
   p.off_O = take(BN * H * p.Ocols * 4);
   p.off_W = take(BN * H * 16);

@@ -1,26 +1,43 @@
 // prologue.cu -- frames to global points and the lifted Q / K / V rows (HBM-bound).
 //
-// One CTA per (128-residue tile, sample).  The CTA first reduces the tile's
-// origin o_T (mean translation of its valid residues), then one warp per
-// residue applies the frame T_i(x) = R_i x + t_i ("Required behavior": frames,
-// column-vector convention) to every query/key/value point of every head,
-// expresses the global points relative to o_T, and writes the lifted rows
-// documented in plan.h, with the distance weight folded into the query
-// columns (squared-norm expansion of FlashIPA's lifted attention).
+// Two kernels:
+//   origin: one CTA per (128-residue tile, sample) reduces the origin o_G of
+//           each 32-residue group (mean translation of its valid residues) and
+//           the tile's valid flag;
+//   lift:   one CTA per 8 residues of a sample, all heads.  It stages the
+//           frames, z1 rows and Wb^T in shared memory, applies every frame
+//           T_i(x) = R_i x + t_i (page "Invariant point attention (IPA)",
+//           Required behavior: column-vector convention) to all query / key /
+//           value points in parallel, and then writes every lifted row of
+//           plan.h as 16-byte chunks of 8 fp16 values.  Each column segment is
+//           padded to a multiple of 8, so a chunk never straddles two segments.
+// The distance weight g is folded into the query point columns, following the
+// squared-norm expansion of FlashIPA's lifted attention.
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace fipa {
 namespace {
 
-constexpr int kPrologueWarps = 16;
+constexpr int kLiftRes = 8;        // residues per lift CTA (divides the 128-residue tile)
+constexpr int kLiftThreads = 256;
 
 __device__ __forceinline__ __half hi_half(float x) { return __float2half_rn(x); }
 __device__ __forceinline__ __half lo_half(float x) {
   return __float2half_rn(x - __half2float(__float2half_rn(x)));
 }
-// Part `seg` of a value stored as `pattern`: 0 -> hi, 1 -> lo.
-__device__ __forceinline__ __half part(float x, int is_lo) { return is_lo ? lo_half(x) : hi_half(x); }
+__device__ __forceinline__ uint32_t pack2(float a, float b, bool lo) {
+  const __half x = lo ? lo_half(a) : hi_half(a), y = lo ? lo_half(b) : hi_half(b);
+  return (uint32_t)__half_as_ushort(x) | ((uint32_t)__half_as_ushort(y) << 16);
+}
+__device__ __forceinline__ void store8(__half* dst, const float (&v)[8], bool lo) {
+  uint4 u;
+  u.x = pack2(v[0], v[1], lo);
+  u.y = pack2(v[2], v[3], lo);
+  u.z = pack2(v[4], v[5], lo);
+  u.w = pack2(v[6], v[7], lo);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
 
 struct PrologueArgs {
   Plan p;
@@ -29,8 +46,35 @@ struct PrologueArgs {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(kPrologueWarps * 32)
-fipa_prologue_kernel(const PrologueArgs a) {
+__global__ void __launch_bounds__(kTile) fipa_origin_kernel(const PrologueArgs a) {
+  // warp w reduces 32-residue group 4t+w of the 128-residue tile t
+  const Plan& p = a.p;
+  const T* tr = static_cast<const T*>(a.in.trans);
+  const int t = blockIdx.x, b = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int s_any[kTile / 32];
+  float sx = 0.f, sy = 0.f, sz = 0.f, cnt = 0.f;
+  const int i = t * kTile + threadIdx.x;
+  if (i < p.N && a.in.mask[(size_t)b * p.N + i]) {
+    const size_t o = ((size_t)b * p.N + i) * 3;
+    sx = ld_in(tr, o + 0); sy = ld_in(tr, o + 1); sz = ld_in(tr, o + 2); cnt = 1.f;
+  }
+  for (int off = 16; off; off >>= 1) {
+    sx += __shfl_xor_sync(0xffffffffu, sx, off);
+    sy += __shfl_xor_sync(0xffffffffu, sy, off);
+    sz += __shfl_xor_sync(0xffffffffu, sz, off);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+  }
+  if (lane == 0) {
+    const float inv = cnt > 0.f ? 1.f / cnt : 0.f;
+    a.w.orig[(size_t)b * p.nG + t * 4 + warp] = make_float4(sx * inv, sy * inv, sz * inv, cnt);
+    s_any[warp] = cnt > 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) a.w.flag[(size_t)b * p.nT + t] = (s_any[0] | s_any[1] | s_any[2] | s_any[3]) ? 1 : 0;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueArgs a) {
   const Plan& p = a.p;
   const T* q = static_cast<const T*>(a.in.q);
   const T* k = static_cast<const T*>(a.in.k);
@@ -44,160 +88,207 @@ fipa_prologue_kernel(const PrologueArgs a) {
   const T* z2 = static_cast<const T*>(a.in.z2);
   const T* Wb = static_cast<const T*>(a.in.Wb);
   const T* raw = static_cast<const T*>(a.in.raw);
-
-  const int t = blockIdx.x, b = blockIdx.y;
-  const int N = p.N, H = p.H, P = p.P, Q = p.Q, RCz = p.R * p.Cz;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = p.N, H = p.H, P = p.P, Q = p.Q, Cz = p.Cz, RCz = p.R * p.Cz;
+  const int b = blockIdx.y, i0 = blockIdx.x * kLiftRes;
+  const int nres = min(kLiftRes, N - i0);
+  const int npt = 2 * P + Q;                 // query, key and value points of one head
 
   extern __shared__ float sh[];
-  __shared__ float red[kPrologueWarps][4];
-  __shared__ float4 s_orig;
+  float* wbt = sh;                                   // [H][Cz]  Wb^T / sqrt(3)
+  float* z1s = wbt + H * Cz;                         // [8][R*Cz]
+  float* z2s = z1s + kLiftRes * RCz;                 // [8][R*Cz]
+  float* pts = z2s + kLiftRes * RCz;                 // [8][H][npt][3]  global point - o_G
+  float* frm = pts + kLiftRes * H * npt * 3;         // [8][12]  R (row-major), t - o_G
+  float* qs = frm + kLiftRes * 12;                   // [8][H][D]
+  float* ks = qs + kLiftRes * H * p.D;               // [8][H][D]
+  float* vs = ks + kLiftRes * H * p.D;               // [8][H][Dv]
+  __shared__ float s_gamma[64];
+  __shared__ int s_valid[kLiftRes];
 
-  // ---- tile origin: mean translation of the valid residues of the tile
-  {
-    float sx = 0.f, sy = 0.f, sz = 0.f, cnt = 0.f;
-    if (threadIdx.x < kTile) {
-      const int i = t * kTile + threadIdx.x;
-      if (i < N && a.in.mask[(size_t)b * N + i]) {
-        const size_t o = ((size_t)b * N + i) * 3;
-        sx = ld_in(tr, o + 0); sy = ld_in(tr, o + 1); sz = ld_in(tr, o + 2); cnt = 1.f;
-      }
-    }
-    for (int off = 16; off; off >>= 1) {
-      sx += __shfl_xor_sync(0xffffffffu, sx, off);
-      sy += __shfl_xor_sync(0xffffffffu, sy, off);
-      sz += __shfl_xor_sync(0xffffffffu, sz, off);
-      cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-    }
-    if (lane == 0) { red[warp][0] = sx; red[warp][1] = sy; red[warp][2] = sz; red[warp][3] = cnt; }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      float ax = 0.f, ay = 0.f, az = 0.f, ac = 0.f;
-      for (int wi = 0; wi < kTile / 32; ++wi) { ax += red[wi][0]; ay += red[wi][1]; az += red[wi][2]; ac += red[wi][3]; }
-      const float inv = ac > 0.f ? 1.f / ac : 0.f;
-      s_orig = make_float4(ax * inv, ay * inv, az * inv, ac);
-      a.w.orig[(size_t)b * p.nT + t] = s_orig;
-      a.w.flag[(size_t)b * p.nT + t] = ac > 0.f ? 1 : 0;
-    }
-    __syncthreads();
-  }
-  const float ox = s_orig.x, oy = s_orig.y, oz = s_orig.z;
-
-  // per-warp scratch: a' [P*3], b' [P*3], g' [Q*3], z1 row [R*Cz]
-  const int PQ = P > Q ? P : Q;
-  float* pa = sh + (size_t)warp * (9 * PQ + RCz);
-  float* pb = pa + 3 * PQ;
-  float* pg = pb + 3 * PQ;
-  float* z1s = pg + 3 * PQ;
-  const float sqk = rsqrtf(3.0f * (float)p.D);
+  // ---- stage every input of the 8 residues (independent loads, issued together)
   const float inv_sqrt3 = rsqrtf(3.0f);
+  const size_t bi0 = (size_t)b * N + i0;
+  for (int e = threadIdx.x; e < H * Cz; e += blockDim.x) {
+    const int h = e / Cz, c = e - h * Cz;
+    wbt[e] = ld_in(Wb, (size_t)c * H + h) * inv_sqrt3;
+  }
+#pragma unroll 4
+  for (int e = threadIdx.x; e < nres * RCz; e += blockDim.x) {
+    z1s[e] = ld_in(z1, bi0 * RCz + e);
+    z2s[e] = ld_in(z2, bi0 * RCz + e);
+  }
+#pragma unroll 4
+  for (int e = threadIdx.x; e < nres * H * p.D; e += blockDim.x) {
+    qs[e] = ld_in(q, bi0 * H * p.D + e);
+    ks[e] = ld_in(k, bi0 * H * p.D + e);
+  }
+#pragma unroll 4
+  for (int e = threadIdx.x; e < nres * H * p.Dv; e += blockDim.x) vs[e] = ld_in(v, bi0 * H * p.Dv + e);
+  for (int e = threadIdx.x; e < nres * 12; e += blockDim.x) {
+    const int r = e / 12, c = e - r * 12;
+    const size_t bi = bi0 + r;
+    if (c < 9) {
+      frm[e] = ld_in(rot, bi * 9 + c);
+    } else {
+      const float4 o = a.w.orig[(size_t)b * p.nG + (i0 + r) / kGroup];
+      frm[e] = ld_in(tr, bi * 3 + (c - 9)) - (c == 9 ? o.x : c == 10 ? o.y : o.z);
+    }
+  }
+  for (int h = threadIdx.x; h < H && h < 64; h += blockDim.x) s_gamma[h] = point_weight(ld_in(raw, h), P);
+  if (threadIdx.x < nres) s_valid[threadIdx.x] = a.in.mask[bi0 + threadIdx.x] != 0;
+  __syncthreads();
 
-  for (int r = warp; r < kTile; r += kPrologueWarps) {
-    const int i = t * kTile + r;
-    if (i >= N) break;
+  // ---- every point of every head of the 8 residues, relative to its group origin
+#pragma unroll 4
+  for (int e = threadIdx.x; e < nres * H * npt; e += blockDim.x) {
+    const int r = e / (H * npt), rem = e - r * H * npt, h = rem / npt, pt = rem - h * npt;
+    const size_t bih = ((size_t)b * N + i0 + r) * H + h;
+    const T* src = pt < P ? qp + (bih * P + pt) * 3
+                 : pt < 2 * P ? kp + (bih * P + (pt - P)) * 3 : vp + (bih * Q + (pt - 2 * P)) * 3;
+    const float x0 = ld_in(src, 0), x1 = ld_in(src, 1), x2 = ld_in(src, 2);
+    const float* F = frm + r * 12;
+    float* o = pts + (size_t)e * 3;
+    o[0] = F[0] * x0 + F[1] * x1 + F[2] * x2 + F[9];
+    o[1] = F[3] * x0 + F[4] * x1 + F[5] * x2 + F[10];
+    o[2] = F[6] * x0 + F[7] * x1 + F[8] * x2 + F[11];
+  }
+  __syncthreads();
+
+  // ---- per (residue, head) fp32 corrections (and the fp32 points of float32 mode)
+  for (int e = threadIdx.x; e < nres * H; e += blockDim.x) {
+    const int r = e / H, h = e - r * H;
+    const float g = s_gamma[h < 64 ? h : 63];
+    const float* pa = pts + (size_t)e * npt * 3;
+    const float* pb = pa + 3 * P;
+    float Ax = 0.f, Ay = 0.f, Az = 0.f, a2 = 0.f, Bx = 0.f, By = 0.f, Bz = 0.f, b2 = 0.f;
+    for (int pp = 0; pp < P; ++pp) {
+      Ax += pa[3 * pp]; Ay += pa[3 * pp + 1]; Az += pa[3 * pp + 2];
+      a2 += pa[3 * pp] * pa[3 * pp] + pa[3 * pp + 1] * pa[3 * pp + 1] + pa[3 * pp + 2] * pa[3 * pp + 2];
+      Bx += pb[3 * pp]; By += pb[3 * pp + 1]; Bz += pb[3 * pp + 2];
+      b2 += pb[3 * pp] * pb[3 * pp] + pb[3 * pp + 1] * pb[3 * pp + 1] + pb[3 * pp + 2] * pb[3 * pp + 2];
+    }
+    const bool valid = s_valid[r] != 0;
+    const size_t bhi = ((size_t)b * H + h) * N + i0 + r;
+    if (p.geo_simt) {
+      a.w.kvec[bhi] = make_float4(valid ? 0.f : -INFINITY, 0.f, 0.f, 0.f);
+      a.w.qvec[bhi] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int x = 0; x < 3 * P; ++x) {
+        a.w.QP[bhi * 3 * P + x] = pa[x];
+        a.w.KP[bhi * 3 * P + x] = valid ? pb[x] : 0.f;
+      }
+    } else {
+      a.w.kvec[bhi] = valid ? make_float4(-g * b2, Bx, By, Bz) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+      a.w.qvec[bhi] = make_float4(Ax, Ay, Az, -g * a2);
+    }
+  }
+
+  // ---- every lifted row as 16-byte chunks (8 fp16 values of one segment)
+  const int qc = p.Kq / 8, kc = p.KHp / 8, vc = p.VHp / 8, zc = p.Zp / 8;
+  const int cpr = H * (qc + kc + vc) + zc;          // chunks per residue
+  const float sqk = rsqrtf(3.0f * (float)p.D);
+  for (int e = threadIdx.x; e < nres * cpr; e += blockDim.x) {
+    const int r = e / cpr;
+    int c = e - r * cpr;
+    const int i = i0 + r;
     const size_t bi = (size_t)b * N + i;
-    const bool valid = a.in.mask[bi] != 0;
-    float R[9], tv[3];
+    const bool valid = s_valid[r] != 0;
+    float vals[8];
 #pragma unroll
-    for (int e = 0; e < 9; ++e) R[e] = ld_in(rot, bi * 9 + e);
+    for (int t = 0; t < 8; ++t) vals[t] = 0.f;
+    bool lo = false;
+    __half* dst;
+    if (c < H * qc) {                                  // ---- query row of head h
+      const int h = c / qc, col = (c - h * qc) * 8;
+      dst = a.w.Q + (((size_t)b * H + h) * N + i) * p.Kq + col;
+      if (valid) {
+        if (col < p.KHp) {
+          const int sc = p.nsq * p.D8;
+          if (col < sc) {
+            const int seg = col / p.D8, e0 = col - seg * p.D8;
+            lo = (seg == 2);
 #pragma unroll
-    for (int e = 0; e < 3; ++e) tv[e] = ld_in(tr, bi * 3 + e);
-    const float tx = tv[0] - ox, ty = tv[1] - oy, tz = tv[2] - oz;   // t_i - o_T
-
-    // pair factors of this residue: z2 row goes to Z, z1 row to scratch
-    __half* zrow = a.w.Z + bi * p.Zp;
-    for (int e = lane; e < RCz; e += 32) {
-      z1s[e] = ld_in(z1, bi * RCz + e);
-      const float x = valid ? ld_in(z2, bi * RCz + e) : 0.f;
-      for (int seg = 0; seg < p.nz; ++seg) zrow[seg * RCz + e] = part(x, seg == 1);
-    }
-    for (int c = p.Zc + lane; c < p.Zp; c += 32) zrow[c] = __float2half_rn(0.f);
-    __syncwarp();
-
-    for (int h = 0; h < H; ++h) {
-      const float g = point_weight(ld_in(raw, h), P);
-      const size_t bhi = ((size_t)b * H + h) * N + i;
-      const size_t in_pts = (bi * H + h);
-      // global points relative to the tile origin
-      for (int e = lane; e < PQ; e += 32) {
-        if (e < P) {
-          float x0 = ld_in(qp, (in_pts * P + e) * 3 + 0), x1 = ld_in(qp, (in_pts * P + e) * 3 + 1),
-                x2 = ld_in(qp, (in_pts * P + e) * 3 + 2);
-          pa[e * 3 + 0] = R[0] * x0 + R[1] * x1 + R[2] * x2 + tx;
-          pa[e * 3 + 1] = R[3] * x0 + R[4] * x1 + R[5] * x2 + ty;
-          pa[e * 3 + 2] = R[6] * x0 + R[7] * x1 + R[8] * x2 + tz;
-          x0 = ld_in(kp, (in_pts * P + e) * 3 + 0); x1 = ld_in(kp, (in_pts * P + e) * 3 + 1);
-          x2 = ld_in(kp, (in_pts * P + e) * 3 + 2);
-          pb[e * 3 + 0] = R[0] * x0 + R[1] * x1 + R[2] * x2 + tx;
-          pb[e * 3 + 1] = R[3] * x0 + R[4] * x1 + R[5] * x2 + ty;
-          pb[e * 3 + 2] = R[6] * x0 + R[7] * x1 + R[8] * x2 + tz;
-        }
-        if (e < Q) {
-          const float x0 = ld_in(vp, (in_pts * Q + e) * 3 + 0), x1 = ld_in(vp, (in_pts * Q + e) * 3 + 1),
-                      x2 = ld_in(vp, (in_pts * Q + e) * 3 + 2);
-          pg[e * 3 + 0] = R[0] * x0 + R[1] * x1 + R[2] * x2 + tx;
-          pg[e * 3 + 1] = R[3] * x0 + R[4] * x1 + R[5] * x2 + ty;
-          pg[e * 3 + 2] = R[6] * x0 + R[7] * x1 + R[8] * x2 + tz;
-        }
-      }
-      __syncwarp();
-
-      // ---- lifted query row
-      __half* qrow = a.w.Q + bhi * p.Kq;
-      const float vs = valid ? 1.f : 0.f;
-      for (int seg = 0; seg < p.nsq; ++seg)
-        for (int d = lane; d < p.D; d += 32)
-          qrow[seg * p.D + d] = part(vs * ld_in(q, in_pts * p.D + d) * sqk, seg == 2);
-      {
-        const int base = p.nsq * p.D, n3 = 3 * P;
-        for (int seg = 0; seg < 3; ++seg)
-          for (int e = lane; e < n3; e += 32) qrow[base + seg * n3 + e] = part(vs * 2.f * g * pa[e], seg == 2);
-        for (int c = p.KHc + lane; c < p.KHp; c += 32) qrow[c] = __float2half_rn(0.f);
-      }
-      for (int seg = 0; seg < p.nz; ++seg)
-        for (int rr = 0; rr < p.R; ++rr)
-          for (int c = lane; c < p.Cz; c += 32) {
-            const float u = vs * z1s[rr * p.Cz + c] * ld_in(Wb, (size_t)c * H + h) * inv_sqrt3;
-            qrow[p.KHp + seg * RCz + rr * p.Cz + c] = part(u, seg == 2);
+            for (int t = 0; t < 8; ++t)
+              if (e0 + t < p.D) vals[t] = qs[(r * H + h) * p.D + e0 + t] * sqk;
+          } else if (!p.geo_simt && col < sc + 3 * p.P38) {
+            const int seg = (col - sc) / p.P38, e0 = col - sc - seg * p.P38;
+            const float g2 = 2.f * s_gamma[h < 64 ? h : 63];
+            const float* pa = pts + ((size_t)r * H + h) * npt * 3;
+            lo = (seg == 2);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              if (e0 + t < 3 * P) vals[t] = g2 * pa[e0 + t];
           }
-      for (int c = p.KHp + p.Zc + lane; c < p.Kq; c += 32) qrow[c] = __float2half_rn(0.f);
-
-      // ---- lifted key row (head part)
-      __half* krow = a.w.KH + bhi * p.KHp;
-      for (int seg = 0; seg < p.nsq; ++seg)
-        for (int d = lane; d < p.D; d += 32) krow[seg * p.D + d] = part(vs * ld_in(k, in_pts * p.D + d), seg == 1);
-      {
-        const int base = p.nsq * p.D, n3 = 3 * P;
-        for (int seg = 0; seg < 3; ++seg)
-          for (int e = lane; e < n3; e += 32) krow[base + seg * n3 + e] = part(vs * pb[e], seg == 1);
-        for (int c = p.KHc + lane; c < p.KHp; c += 32) krow[c] = __float2half_rn(0.f);
-      }
-
-      // ---- lifted value row (head part)
-      __half* vrow = a.w.VH + bhi * p.VHp;
-      for (int seg = 0; seg < p.nsv; ++seg)
-        for (int d = lane; d < p.Dv; d += 32) vrow[seg * p.Dv + d] = part(vs * ld_in(v, in_pts * p.Dv + d), seg == 1);
-      {
-        const int base = p.nsv * p.Dv, n3 = 3 * Q;
-        for (int seg = 0; seg < 2; ++seg)
-          for (int e = lane; e < n3; e += 32) vrow[base + seg * n3 + e] = part(vs * pg[e], seg == 1);
-        for (int c = p.VHc + lane; c < p.VHp; c += 32) vrow[c] = __float2half_rn(0.f);
-      }
-
-      // ---- per-key and per-query fp32 corrections
-      if (lane == 0) {
-        float Ax = 0.f, Ay = 0.f, Az = 0.f, a2 = 0.f, Bx = 0.f, By = 0.f, Bz = 0.f, b2 = 0.f;
-        for (int e = 0; e < P; ++e) {
-          Ax += pa[3 * e]; Ay += pa[3 * e + 1]; Az += pa[3 * e + 2];
-          a2 += pa[3 * e] * pa[3 * e] + pa[3 * e + 1] * pa[3 * e + 1] + pa[3 * e + 2] * pa[3 * e + 2];
-          Bx += pb[3 * e]; By += pb[3 * e + 1]; Bz += pb[3 * e + 2];
-          b2 += pb[3 * e] * pb[3 * e] + pb[3 * e + 1] * pb[3 * e + 1] + pb[3 * e + 2] * pb[3 * e + 2];
+        } else {
+          int cc = col - p.KHp, e0;
+          if (p.nqz == 2) {                          // [u hi | u lo], each Zp wide
+            lo = cc >= p.Zp;
+            e0 = lo ? cc - p.Zp : cc;
+          } else {                                   // [u hi | u hi | u lo], RC8 apart
+            const int seg = cc / p.RC8;
+            e0 = seg < p.nz ? cc - seg * p.RC8 : RCz;
+            lo = (seg == 2);
+          }
+          int rr = e0 / Cz, c0 = e0 - rr * Cz;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            if (e0 + t < RCz) vals[t] = z1s[r * RCz + e0 + t] * wbt[h * Cz + c0];
+            if (++c0 == Cz) { c0 = 0; ++rr; }
+          }
         }
-        a.w.kvec[bhi] = valid ? make_float4(-g * b2, Bx, By, Bz) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
-        a.w.qvec[bhi] = make_float4(Ax, Ay, Az, -g * a2);
       }
-      __syncwarp();
+    } else if ((c -= H * qc) < H * kc) {               // ---- key row (head part)
+      const int h = c / kc, col = (c - h * kc) * 8;
+      dst = a.w.KH + (((size_t)b * H + h) * N + i) * p.KHp + col;
+      const int sc = p.nsq * p.D8;
+      if (valid) {
+        if (col < sc) {
+          const int seg = col / p.D8, e0 = col - seg * p.D8;
+          lo = (seg == 1);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (e0 + t < p.D) vals[t] = ks[(r * H + h) * p.D + e0 + t];
+        } else if (!p.geo_simt && col < sc + 3 * p.P38) {
+          const int seg = (col - sc) / p.P38, e0 = col - sc - seg * p.P38;
+          const float* pb = pts + ((size_t)r * H + h) * npt * 3 + 3 * P;
+          lo = (seg == 1);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (e0 + t < 3 * P) vals[t] = pb[e0 + t];
+        }
+      }
+    } else if ((c -= H * kc) < H * vc) {               // ---- value row (head part)
+      const int h = c / vc, col = (c - h * vc) * 8;
+      dst = a.w.VH + (((size_t)b * H + h) * N + i) * p.VHp + col;
+      const int sc = p.nsv * p.Dv8;
+      if (valid) {
+        if (col < sc) {
+          const int seg = col / p.Dv8, e0 = col - seg * p.Dv8;
+          lo = (seg == 1);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (e0 + t < p.Dv) vals[t] = vs[(r * H + h) * p.Dv + e0 + t];
+        } else if (col < sc + 2 * p.Q38) {
+          const int seg = (col - sc) / p.Q38, e0 = col - sc - seg * p.Q38;
+          const float* pg = pts + ((size_t)r * H + h) * npt * 3 + 6 * P;
+          lo = (seg == 1);
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            if (e0 + t < 3 * Q) vals[t] = pg[e0 + t];
+        }
+      }
+    } else {                                           // ---- pair factor row z2 (shared by heads)
+      c -= H * vc;
+      const int col = c * 8;
+      dst = a.w.Z + bi * p.Zp + col;
+      const int seg = col / p.RC8, e0 = col - seg * p.RC8;
+      if (valid && seg < p.nz) {
+        lo = (seg == 1);
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+          if (e0 + t < RCz) vals[t] = z2s[r * RCz + e0 + t];
+      }
     }
+    store8(dst, vals, lo);
   }
 }
 
@@ -205,19 +296,19 @@ fipa_prologue_kernel(const PrologueArgs a) {
 
 cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s) {
   PrologueArgs a{p, in, w};
-  const int PQ = p.P > p.Q ? p.P : p.Q;
-  const size_t smem = (size_t)kPrologueWarps * (9 * PQ + p.R * p.Cz) * sizeof(float);
-  dim3 grid(p.nT, p.B);
+  dim3 g1(p.nT, p.B), g2((p.N + kLiftRes - 1) / kLiftRes, p.B);
   if (p.f32) {
-    auto kfn = fipa_prologue_kernel<float>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    fipa_origin_kernel<float><<<g1, kTile, 0, s>>>(a);
+    auto kfn = fipa_lift_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.lift_smem);
     if (e != cudaSuccess) return e;
-    kfn<<<grid, kPrologueWarps * 32, smem, s>>>(a);
+    kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
   } else {
-    auto kfn = fipa_prologue_kernel<__nv_bfloat16>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    fipa_origin_kernel<__nv_bfloat16><<<g1, kTile, 0, s>>>(a);
+    auto kfn = fipa_lift_kernel<__nv_bfloat16>;
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.lift_smem);
     if (e != cudaSuccess) return e;
-    kfn<<<grid, kPrologueWarps * 32, smem, s>>>(a);
+    kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
   }
   return cudaGetLastError();
 }

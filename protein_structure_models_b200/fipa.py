@@ -64,6 +64,10 @@ def load_library():
     lib.fipa_status_string.restype = ctypes.c_char_p
     lib.fipa_last_error.argtypes = [vp]
     lib.fipa_last_error.restype = ctypes.c_char_p
+    lib.fipa_enable_stage_timing.argtypes = [vp, c_int]
+    lib.fipa_enable_stage_timing.restype = c_int
+    lib.fipa_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), c_int]
+    lib.fipa_stage_times.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -161,6 +165,17 @@ class Fipa:
             ctypes.c_void_p(s.cuda_stream))
         self._check(st)
         return out
+
+    STAGES = ("prologue", "core", "weight_prep", "features", "out_proj", "attention")
+
+    def enable_stage_timing(self, enable: bool = True):
+        self._check(self.lib.fipa_enable_stage_timing(self.handle, 1 if enable else 0))
+
+    def stage_times(self) -> dict:
+        """Device ms of each stage of the most recent timed forward."""
+        buf = (ctypes.c_float * 6)()
+        self._check(self.lib.fipa_stage_times(self.handle, buf, 6))
+        return dict(zip(self.STAGES, [float(x) for x in buf]))
 
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))

@@ -27,16 +27,7 @@ def to_device(inp: dict, dtype: str, device="cuda") -> dict:
     return out
 
 
-def slice_batch(inp: dict, bsel) -> dict:
-    """Inputs restricted to batch elements `bsel` (samples are independent)."""
-    out = dict(inp)
-    for k in FLOAT_KEYS + ("mask",):
-        if k in ("Wb", "point_weight_raw", "w_out", "b_out"):
-            continue
-        out[k] = inp[k][bsel]
-    if inp.get("pair_mask") is not None:
-        out["pair_mask"] = inp["pair_mask"][bsel]
-    return out
+from workloads import slice_batch  # noqa: E402,F401  (re-exported for the tests)
 
 
 def max_err(a, b):

@@ -24,7 +24,7 @@ from typing import Optional
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "round_to_dtype",
-           "random_rotations", "SWEEP_N", "BASE_SEED"]
+           "random_rotations", "slice_batch", "SWEEP_N", "BASE_SEED"]
 
 BASE_SEED = 20261202
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)
@@ -208,4 +208,18 @@ def make_inputs(wl: Workload, seed: Optional[int] = None) -> dict:
             pair_mask[b, i_star, :] = False
     out["pair_mask"] = pair_mask
     out["eps"] = 1e-8
+    return out
+
+
+_PER_SAMPLE = ("q", "k", "v", "q_points", "k_points", "v_points", "rotation", "translation",
+               "z1", "z2", "mask")
+
+
+def slice_batch(inp: dict, bsel) -> dict:
+    """The inputs restricted to batch elements `bsel` (samples are independent)."""
+    out = dict(inp)
+    for key in _PER_SAMPLE:
+        out[key] = inp[key][bsel]
+    if inp.get("pair_mask") is not None:
+        out["pair_mask"] = inp["pair_mask"][bsel]
     return out
