@@ -137,11 +137,27 @@ fipa_status fipa_sync_status(fipa_handle* h, void* stream);
 fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable);
 
 /* Device time in milliseconds of each stage of the most recent fipa_forward
- * recorded with stage timing on, in launch order: [0] prologue, [1] fused
- * attention core, [2] output-weight preparation, [3] features, [4] output
- * projection, [5] attention output (0 when not requested).  Waits for that
- * call's last event.  `n` = capacity of `ms` (up to 6 values are written). */
+ * recorded with stage timing on, in launch order: [0] prologue (tile origins
+ * and lifted rows), [1] fused attention core with the feature epilogue,
+ * [2] output-weight preparation, [3] output projection, [4] attention output
+ * (0 when not requested).  Waits for that call's last event.  `n` = capacity
+ * of `ms` (up to 5 values are written). */
 fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n);
+
+/* Debug tracing.  When the environment variable FIPA_TRACE_CTA=<n> is set at
+ * fipa_create, the handle owns a small device buffer and the fused core's CTA
+ * number n (linear block index) logs (event id, SM clock) pairs per warp role
+ * during every fipa_forward.  fipa_trace_copy waits for `stream` and copies the
+ * log: 4 roles (0 TMA producer, 1 MMA issuer, 2 softmax lane 0, 3 key-term
+ * warps) x FIPA_TRACE_CAP entries x {event, clock}, int64, -1 = unused.
+ * Returns FIPA_ERR_INVALID_ARG if tracing is off or `n_values` is too small. */
+#define FIPA_TRACE_CAP 4096
+fipa_status fipa_trace_copy(fipa_handle* h, int64_t* host, size_t n_values, void* stream);
+
+/* Number of kernels one fipa_forward with these dims launches (plus one when
+ * the attention output is requested).  Pure host arithmetic. */
+fipa_status fipa_kernel_count(const fipa_handle* h, const fipa_dims* dims, int with_attention,
+                              int* count);
 
 /* Static description of a status code. */
 const char* fipa_status_string(fipa_status s);

@@ -122,8 +122,7 @@ cudaError_t launch_attention_dump(const Plan& p, const Inputs& in, const Work& w
   AttnArgs a{p, w.Q, w.KH, w.Z, w.kvec, w.qvec, w.orig, w.stats, w.QP, w.KP, in.mask, in.pair_mask, in.raw,
              out.attention};
   const size_t smem = (size_t)kRows * p.Kq * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(fipa_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_attention_kernel));
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)p.H, (unsigned)p.B);
   fipa_attention_kernel<<<grid, 128, smem, s>>>(a);

@@ -42,12 +42,19 @@ struct CoreArgs {
   const uint8_t* mask;
   const uint8_t* pair_mask;
   const void* raw;
-  float* O;
-  float4* W;
+  const void* rot;
+  const void* trans;
+  const void* z1;
+  __half* feat;
+  uint8_t* rowflag;
+  float* local_points;
+  float eps;
   float2* stats;
   float* lse;
   int* status;
   unsigned long long timeout_ns;
+  long long* trace;
+  int trace_cta;
 };
 
 // Shared-memory tail after the Qhat tile and the ring (byte offsets).
@@ -70,6 +77,150 @@ constexpr int kKpBuf = 7168;       // fp32 key points of two key tiles (float32-
 __device__ __forceinline__ float load_raw(const CoreArgs& a, int h) {
   return a.p.f32 ? static_cast<const float*>(a.raw)[h]
                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.raw)[h]);
+}
+
+__device__ __forceinline__ float ld_any(const void* ptr, size_t i, int f32) {
+  return f32 ? __ldg(static_cast<const float*>(ptr) + i)
+             : __bfloat162float(static_cast<const __nv_bfloat16*>(ptr)[i]);
+}
+
+__device__ __forceinline__ uint32_t half2_bits(__half a, __half b) {
+  return (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+}
+
+// Feature values val(0..n-1) at feature columns [col, col+n) of the projection
+// operand row: fp16 hi at col and lo at F+col (float32 inputs: hi, hi, lo at
+// col, F+col, 2F+col).  16-byte stores where the run is aligned.
+template <typename Fn>
+__device__ __forceinline__ void put_run(__half* frow, int F, int f32, int col, int n, Fn&& val) {
+  for (int k0 = 0; k0 < n; k0 += 8) {
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = k0 + t < n ? val(k0 + t) : 0.f;
+    __half hi[8], lo[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      hi[t] = __float2half_rn(v[t]);
+      lo[t] = __float2half_rn(v[t] - __half2float(hi[t]));
+    }
+    const int c = col + k0;
+    if (k0 + 8 <= n && (c & 7) == 0 && (F & 7) == 0) {
+      const uint4 H4 = make_uint4(half2_bits(hi[0], hi[1]), half2_bits(hi[2], hi[3]), half2_bits(hi[4], hi[5]),
+                                  half2_bits(hi[6], hi[7]));
+      const uint4 L4 = make_uint4(half2_bits(lo[0], lo[1]), half2_bits(lo[2], lo[3]), half2_bits(lo[4], lo[5]),
+                                  half2_bits(lo[6], lo[7]));
+      *reinterpret_cast<uint4*>(frow + c) = H4;
+      if (f32) {
+        *reinterpret_cast<uint4*>(frow + F + c) = H4;
+        *reinterpret_cast<uint4*>(frow + 2 * F + c) = L4;
+      } else {
+        *reinterpret_cast<uint4*>(frow + F + c) = L4;
+      }
+    } else {
+      for (int t = 0; t < 8 && k0 + t < n; ++t) {
+        frow[c + t] = hi[t];
+        if (f32) { frow[F + c + t] = hi[t]; frow[2 * F + c + t] = lo[t]; }
+        else     { frow[F + c + t] = lo[t]; }
+      }
+    }
+  }
+}
+
+// 32 feature values from registers at columns [col, col+32), as put_run.
+__device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col, const float (&v)[32]) {
+#pragma unroll
+  for (int k0 = 0; k0 < 32; k0 += 8) {
+    __half hi[8], lo[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      hi[t] = __float2half_rn(v[k0 + t]);
+      lo[t] = __float2half_rn(v[k0 + t] - __half2float(hi[t]));
+    }
+    const int c = col + k0;
+    if ((c & 7) == 0 && (F & 7) == 0) {
+      const uint4 H4 = make_uint4(half2_bits(hi[0], hi[1]), half2_bits(hi[2], hi[3]), half2_bits(hi[4], hi[5]),
+                                  half2_bits(hi[6], hi[7]));
+      const uint4 L4 = make_uint4(half2_bits(lo[0], lo[1]), half2_bits(lo[2], lo[3]), half2_bits(lo[4], lo[5]),
+                                  half2_bits(lo[6], lo[7]));
+      *reinterpret_cast<uint4*>(frow + c) = H4;
+      if (f32) {
+        *reinterpret_cast<uint4*>(frow + F + c) = H4;
+        *reinterpret_cast<uint4*>(frow + 2 * F + c) = L4;
+      } else {
+        *reinterpret_cast<uint4*>(frow + F + c) = L4;
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        frow[c + t] = hi[t];
+        if (f32) { frow[F + c + t] = hi[t]; frow[2 * F + c + t] = lo[t]; }
+        else     { frow[F + c + t] = lo[t]; }
+      }
+    }
+  }
+}
+
+// Features of residue bi for head h (page "Invariant point attention (IPA)",
+// Required behavior): scalar block; local point = R_i^T (sum_j a_ij g_j - t_i),
+// its length sqrt(|local|^2 + eps); pair block; all zero for an empty
+// neighbourhood.  orow = this row's O accumulator divided by l (staged in
+// shared memory); (Gx,Gy,Gz) = sum_j a_ij o_G(j), the group-origin part of
+// the aggregated value points.  Also writes local_points.
+__device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, float* orow, float Gx, float Gy,
+                               float Gz, bool with_pair) {
+  const Plan& p = a.p;
+  const int H = p.H, Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.F;
+  __half* frow = a.feat + bi * p.Kgp;
+  float* lp = a.local_points + (bi * H + h) * (size_t)Q * 3;
+  if (h == 0)
+    for (int c = p.Kg; c < p.Kgp; ++c) frow[c] = __float2half_rn(0.f);
+  const int sc = h * Dv, xc = H * Dv + h * Q, pc = H * Dv + 4 * H * Q + h * Cz;
+  if (empty) {
+    auto zero = [](int) { return 0.f; };
+    put_run(frow, F, p.f32, sc, Dv, zero);
+    for (int blk = 0; blk < 4; ++blk) put_run(frow, F, p.f32, xc + blk * H * Q, Q, zero);
+    if (with_pair) put_run(frow, F, p.f32, pc, Cz, zero);
+    for (int e = 0; e < 3 * Q; ++e) lp[e] = 0.f;
+    return;
+  }
+  float R[9], t[3];
+#pragma unroll
+  for (int e = 0; e < 9; ++e) R[e] = ld_any(a.rot, bi * 9 + e, p.f32);
+#pragma unroll
+  for (int e = 0; e < 3; ++e) t[e] = ld_any(a.trans, bi * 3 + e, p.f32);
+  // scalar block
+  put_run(frow, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
+  // points: aggregate (hi + lo halves + group-origin part), back into the query
+  // frame; the local coordinates overwrite the consumed hi slots, the lengths the lo slots
+  const int gofs = p.nsv * p.Dv8;
+  for (int q = 0; q < Q; ++q) {
+    const float gx = orow[gofs + 3 * q + 0] + orow[gofs + p.Q38 + 3 * q + 0] + Gx - t[0];
+    const float gy = orow[gofs + 3 * q + 1] + orow[gofs + p.Q38 + 3 * q + 1] + Gy - t[1];
+    const float gz = orow[gofs + 3 * q + 2] + orow[gofs + p.Q38 + 3 * q + 2] + Gz - t[2];
+    const float lx = R[0] * gx + R[3] * gy + R[6] * gz;
+    const float ly = R[1] * gx + R[4] * gy + R[7] * gz;
+    const float lz = R[2] * gx + R[5] * gy + R[8] * gz;
+    orow[gofs + 3 * q + 0] = lx;
+    orow[gofs + 3 * q + 1] = ly;
+    orow[gofs + 3 * q + 2] = lz;
+    orow[gofs + p.Q38 + q] = sqrtf(lx * lx + ly * ly + lz * lz + a.eps);
+    lp[3 * q + 0] = lx; lp[3 * q + 1] = ly; lp[3 * q + 2] = lz;
+  }
+  for (int x = 0; x < 3; ++x)
+    put_run(frow, F, p.f32, xc + x * H * Q, Q, [&](int q) { return orow[gofs + 3 * q + x]; });
+  put_run(frow, F, p.f32, xc + 3 * H * Q, Q, [&](int q) { return orow[gofs + p.Q38 + q]; });
+  // pair block through the factors (the tensor-memory path writes it otherwise)
+  if (!with_pair) return;
+  const int RCz = p.R * Cz;
+  put_run(frow, F, p.f32, pc, Cz, [&](int c) {
+    float acc = 0.f;
+    for (int rr = 0; rr < p.R; ++rr) {
+      float u = orow[p.VHp + rr * Cz + c];
+      if (p.f32) u += orow[p.VHp + p.RC8 + rr * Cz + c];
+      acc = fmaf(ld_any(a.z1, bi * RCz + rr * Cz + c, p.f32), u, acc);
+    }
+    return acc;
+  });
 }
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight work).
@@ -149,6 +300,12 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const int nkt = *ntiles;
   const WaitCtx wc{abort_flag, a.status, a.timeout_ns};
+  const int lin_cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  long long* tbase = (a.trace != nullptr && lin_cta == a.trace_cta) ? a.trace : nullptr;
+  auto tracer = [&](int role) { return Tracer{tbase ? tbase + (size_t)role * 2 * kTraceCap : nullptr, 0}; };
+  // per-row softmax state, read by the fused feature epilogue after the roles end
+  float rowM = -INFINITY, rowL = 0.f, rowW[3] = {0.f, 0.f, 0.f};
+  bool row_ok = false;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -163,11 +320,14 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       uint32_t ph = 0;
       bool ok = true;
       uint32_t issued = 0;
+      Tracer tr = tracer(0);
       auto push = [&](const CUtensorMap* tm, int c0, int c1, int c2) {
         if (!ok) return;
+        tr.ev(1);
         if (!mbar_wait(&empty[st], ph ^ 1u, wc, 1)) { ok = false; return; }
         mbar_arrive_expect_tx(&full[st], kChunkBytes);
         tma_load_3d(sRing + st * kChunkBytes, tm, &full[st], c0, c1, c2);
+        tr.ev(2);
         ++issued;
         if (++st == p.nst) { st = 0; ph ^= 1u; }
       };
@@ -197,7 +357,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && nkt > 0) {
+      Tracer tr = tracer(1);
       bool ok = mbar_wait(q_full, 0, wc, 2);
+      tr.ev(10);
       tc_fence_after();
       int st = 0;
       uint32_t ph = 0;
@@ -210,7 +372,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         // last, so the small pair terms accumulate before the large point terms
         const int nb = p.nZ + p.nKH;
         for (int c = 0; c < nb; ++c) {
+          tr.ev(11);
           if (!mbar_wait(&full[st], ph, wc, 3)) return false;
+          tr.ev(12);
           tc_fence_after();
           const uint32_t b0 = sRa + st * kChunkBytes;
           const bool pair = c < p.nZ;
@@ -227,12 +391,15 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           if (++st == p.nst) { st = 0; ph ^= 1u; }
         }
         tc_commit(s_full);
+        tr.ev(17);
         return true;
       };
       auto mma_pv = [&](int s) -> bool {
         const int nchunk = p.nVH + p.nZV;
         for (int c = 0; c < nchunk; ++c) {
+          tr.ev(11);
           if (!mbar_wait(&full[st], ph, wc, 4)) return false;
+          tr.ev(12);
           tc_fence_after();
           const uint32_t b0 = sRa + st * kChunkBytes;
           const uint32_t dcol = tmem + (uint32_t)(p.tmemO + c * kChunk);
@@ -246,16 +413,21 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           if (++st == p.nst) { st = 0; ph ^= 1u; }
         }
         tc_commit(pv_done);
+        tr.ev(18);
         return true;
       };
       if (ok) ok = mma_qk();
       for (int s = 0; ok && s < nkt; ++s) {
         if (s + 1 < nkt) {
+          tr.ev(13);
           if (!mbar_wait(s_free, s & 1, wc, 5)) break;
+          tr.ev(14);
           tc_fence_after();
           if (!mma_qk()) break;
         }
+        tr.ev(15);
         if (!mbar_wait(p_full, s & 1, wc, 6)) break;
+        tr.ev(16);
         tc_fence_after();
         if (!mma_pv(s)) break;
       }
@@ -269,6 +441,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // absent key), D_sj = origin of query group s - origin of key j's group; the
     // four key-group origins of the tile go to shared memory as well.
     const int tt = threadIdx.x - 64;
+    Tracer ktr = tracer(3);
     const float g = point_weight(load_raw(a, h), p.P);
     float4 oq[4];
 #pragma unroll
@@ -277,6 +450,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int kb = s & 1;
       const bool okw = mbar_wait(&kt_empty[kb], ((s >> 1) & 1) ^ 1, wc, 10);
       if (!__all_sync(0xffffffffu, okw)) break;
+      if (tt == 0) ktr.ev(30);
       const int kt = tiles[s];
       if (tt < 4) okbuf[kb * 4 + tt] = a.orig[(size_t)b * p.nG + kt * 4 + tt];
       for (int e = tt; e < kTile; e += 64) {
@@ -299,6 +473,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int e = tt; e < kTile * P3; e += 64) kpb[e] = (size_t)e < lim ? a.KP[base + e] : 0.f;
       }
       mbar_arrive(&kt_full[kb]);
+      if (tt == 0) ktr.ev(31);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
@@ -317,11 +492,15 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint8_t* pmrow = (a.pair_mask != nullptr && in_range) ? a.pair_mask + ((size_t)b * N + i) * N : nullptr;
     float M = -INFINITY, l = 0.f, Wx = 0.f, Wy = 0.f, Wz = 0.f;
     bool ok = true;
+    Tracer str = tracer(2);
+    if (threadIdx.x != 128) str.buf = nullptr;
     for (int s = 0; s < nkt; ++s) {
       const int kt = tiles[s];
       const int kb = s & 1;
 
+      str.ev(20);
       ok = mbar_wait(s_full, s & 1, wc, 7);
+      str.ev(21);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[4][32];
@@ -332,9 +511,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(s_free);
+      str.ev(22);
 
       ok = mbar_wait(&kt_full[kb], (s >> 1) & 1, wc, 11);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      str.ev(23);
       float4 okg[4];
       float rc[4];
 #pragma unroll
@@ -421,11 +602,19 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           const float p1 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 1]), kLog2e, -mb));
           const float p2 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 2]), kLog2e, -mb));
           const float p3 = ex2_approx(fmaf(__uint_as_float(sv[t][e + 3]), kLog2e, -mb));
-          rs0 += p0 + p1;
-          rs1 += p2 + p3;
           const int w = (t & 1) * 16 + e / 2;
           pk[t >> 1][w] = pack_half2(p0, p1);
           pk[t >> 1][w + 1] = pack_half2(p2, p3);
+          if (!SPLIT) {
+            // normalise with the sum of the fp16 weights the P.V product uses
+            const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&pk[t >> 1][w]));
+            const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&pk[t >> 1][w + 1]));
+            rs0 += f01.x + f01.y;
+            rs1 += f23.x + f23.y;
+          } else {
+            rs0 += p0 + p1;
+            rs1 += p2 + p3;
+          }
           if (SPLIT) {
             const __half2 h01 = *reinterpret_cast<const __half2*>(&pk[t >> 1][w]);
             const __half2 h23 = *reinterpret_cast<const __half2*>(&pk[t >> 1][w + 1]);
@@ -439,11 +628,13 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       }
 
       // P and O are free once the previous P.V product has finished
+      str.ev(24);
       if (s > 0) {
         ok = mbar_wait(pv_done, (s - 1) & 1, wc, 8);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
+      str.ev(25);
       if (__any_sync(0xffffffffu, resc)) {
         const float f = resc ? alpha : 1.f;
         for (int c = 0; c < p.Ocols; c += 32) {
@@ -464,32 +655,108 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full);
+      str.ev(26);
     }
     if (ok && nkt > 0) {
       ok = mbar_wait(pv_done, (nkt - 1) & 1, wc, 9);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    if (ok && nkt > 0) {
-      float* orow = a.O + (((size_t)b * N + i) * p.H + h) * p.Ocols;
-      for (int c = 0; c < p.Ocols; c += 32) {
+    rowM = M; rowL = l; rowW[0] = Wx; rowW[1] = Wy; rowW[2] = Wz;
+    row_ok = ok;
+  }
+
+  // ------------------------------------------------- fused feature epilogue
+  // Every MMA has finished and every TMA load has landed, so the Qhat and ring
+  // shared memory is reused to stage each row's value-head accumulators (row
+  // stride +1 float: conflict-free).  Each softmax thread then builds the
+  // features of its (residue, head): the page's scalar block, the aggregated
+  // global points taken back into the query frame, their lengths, and the pair
+  // block through the factors, sum_r z1[i,r,c] U[r,c].
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 4 && *abort_flag == 0) {
+    const int wq = warp - 4;
+    const int r = wq * 32 + lane;
+    const int i = qt * kTile + r;
+    const bool in_range = i < N;
+    const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+    const bool fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(a.z1) & 15) == 0;
+    const int staged = fast_pair ? p.VHp : p.Ocols;         // columns staged in shared memory
+    float* orow = reinterpret_cast<float*>(smem) + (size_t)r * (staged + 1);
+    const float inv = rowL > 0.f ? 1.f / rowL : 0.f;
+    const bool live = row_ok && nkt > 0;
+    if (live) {
+      for (int c = 0; c < staged; c += 32) {
         uint32_t o[32];
         tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
         tmem_ld_wait();
-        if (in_range) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(orow + c + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
-        }
+        for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv;
       }
     }
+    const size_t bi = (size_t)b * N + (in_range ? i : 0);
+    const bool empty = !(rowL > 0.f) || !live;
     if (in_range) {
-      a.W[((size_t)b * N + i) * p.H + h] = make_float4(Wx * inv, Wy * inv, Wz * inv, l);
-      a.stats[(size_t)bh * N + i] = make_float2(M, l);
-      if (a.lse != nullptr) a.lse[(size_t)bh * N + i] = l > 0.f ? (M + log2f(l)) * kLn2 + qv.w : -INFINITY;
+      a.stats[(size_t)bh * N + i] = make_float2(rowM, rowL);
+      if (a.lse != nullptr) {
+        const float4 qv = a.qvec[(size_t)bh * N + i];
+        a.lse[(size_t)bh * N + i] = rowL > 0.f ? (rowM + log2f(rowL)) * kLn2 + qv.w : -INFINITY;
+      }
+      if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
+      write_features(a, bi, h, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair);
+    }
+    if (fast_pair) {
+      // pair block straight from tensor memory, 32 channels at a time
+      const int Cz = p.Cz, RCz = p.R * Cz, pcol = p.H * p.Dv + 4 * p.H * p.Q + h * Cz;
+      __half* frow = a.feat + bi * p.Kgp;
+      for (int c0 = 0; c0 < Cz; c0 += 32) {
+        float acc[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+        for (int rr = 0; rr < p.R; ++rr) {
+          uint32_t o[32];
+          if (live) {
+            tmem_ld32(trow + (uint32_t)(p.tmemO + p.VHp + rr * Cz + c0), o);
+            tmem_ld_wait();
+            if (p.f32) {
+              uint32_t o2[32];
+              tmem_ld32(trow + (uint32_t)(p.tmemO + p.VHp + p.RC8 + rr * Cz + c0), o2);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) + __uint_as_float(o2[e]));
+            }
+          }
+          if (in_range && !empty) {
+            const size_t zoff = bi * RCz + (size_t)rr * Cz + c0;
+            float zv[32];
+            if (p.f32) {
+              const float4* z4 = reinterpret_cast<const float4*>(static_cast<const float*>(a.z1) + zoff);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const float4 t4 = __ldg(z4 + k);
+                zv[4 * k] = t4.x; zv[4 * k + 1] = t4.y; zv[4 * k + 2] = t4.z; zv[4 * k + 3] = t4.w;
+              }
+            } else {
+              const uint4* z4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z1) + zoff);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint4 t4 = __ldg(z4 + k);
+                const uint32_t w4[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                  zv[8 * k + 2 * m] = __uint_as_float(w4[m] << 16);
+                  zv[8 * k + 2 * m + 1] = __uint_as_float(w4[m] & 0xffff0000u);
+                }
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv, acc[e]);
+          }
+        }
+        if (in_range) put_run32(frow, p.F, p.f32, pcol + c0, acc);
+      }
     }
   }
 
@@ -512,17 +779,20 @@ cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Ou
   a.p = p;
   a.kvec = w.kvec; a.qvec = w.qvec; a.QP = w.QP; a.KP = w.KP; a.orig = w.orig; a.flag = w.flag;
   a.mask = in.mask; a.pair_mask = in.pair_mask; a.raw = in.raw;
-  a.O = w.O; a.W = w.W; a.stats = w.stats; a.lse = out.lse;
+  a.rot = in.rot; a.trans = in.trans; a.z1 = in.z1; a.feat = w.feat; a.rowflag = w.rowflag;
+  a.local_points = out.local_points; a.eps = in.eps;
+  a.stats = w.stats; a.lse = out.lse;
   a.status = ctl.status; a.timeout_ns = ctl.timeout_ns;
+  a.trace = ctl.trace; a.trace_cta = ctl.trace_cta;
   dim3 grid(p.nT, p.H, p.B);
   if (p.f32) {
     auto kfn = fipa_core_kernel<true>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.core_smem);
+    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
     if (e != cudaSuccess) return e;
     kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);
   } else {
     auto kfn = fipa_core_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.core_smem);
+    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
     if (e != cudaSuccess) return e;
     kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);
   }

@@ -1,4 +1,4 @@
-// epilogue.cu -- features and the affine output projection.
+// epilogue.cu -- the affine output projection (features are built by the core).
 //
 // Page "Invariant point attention (IPA)", Required behavior:
 //   local_points_ihp = R_i^T (sum_j a_hij T_j(v_jhp) - t_i), zero for an empty
@@ -13,116 +13,49 @@
 namespace fipa {
 namespace {
 
-constexpr int kFeatWarps = 8;
-
-struct FeatArgs {
-  Plan p;
-  const void* rot;
-  const void* trans;
-  const void* z1;
-  const float* O;
-  const float4* W;
-  __half* feat;
-  uint8_t* rowflag;
-  float* local_points;
-  float eps;
-};
-
-// store feature value f at feature index `col` as its 16-bit parts
-__device__ __forceinline__ void put_feature(__half* row, int F, int f32, int col, float f) {
-  const __half hi = __float2half_rn(f);
-  const __half lo = __float2half_rn(f - __half2float(hi));
-  row[col] = hi;
-  if (f32) { row[F + col] = hi; row[2 * F + col] = lo; }
-  else     { row[F + col] = lo; }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(kFeatWarps * 32) fipa_features_kernel(const FeatArgs a) {
-  const Plan& p = a.p;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t bi = (size_t)blockIdx.x * kFeatWarps + warp;     // residue index b*N + i
-  if (bi >= (size_t)p.B * p.N) return;
-  const T* rot = static_cast<const T*>(a.rot);
-  const T* tr = static_cast<const T*>(a.trans);
-  const T* z1 = static_cast<const T*>(a.z1);
-  const int H = p.H, Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.F, RCz = p.R * Cz;
-  __half* frow = a.feat + bi * p.Kgp;
-  float* lrow = a.local_points + bi * (size_t)H * Q * 3;
-
-  const bool empty = !(a.W[bi * H].w > 0.f);     // same neighbourhood for every head
-  if (lane == 0) a.rowflag[bi] = empty ? 0 : 1;
-  if (empty) {
-    for (int c = lane; c < p.Kgp; c += 32) frow[c] = __float2half_rn(0.f);
-    for (int e = lane; e < H * Q * 3; e += 32) lrow[e] = 0.f;
-    return;
-  }
-  for (int c = p.Kg + lane; c < p.Kgp; c += 32) frow[c] = __float2half_rn(0.f);
-  float R[9], t[3];
-#pragma unroll
-  for (int e = 0; e < 9; ++e) R[e] = ld_in(rot, bi * 9 + e);
-#pragma unroll
-  for (int e = 0; e < 3; ++e) t[e] = ld_in(tr, bi * 3 + e);
-  const int gofs = p.nsv * p.Dv8;
-  for (int h = 0; h < H; ++h) {
-    const float* orow = a.O + (bi * H + h) * p.Ocols;
-    const float4 Wv = a.W[bi * H + h];
-    // scalar block
-    for (int d = lane; d < Dv; d += 32) {
-      float s = orow[d];
-      if (p.f32) s += orow[p.Dv8 + d];
-      put_feature(frow, F, p.f32, h * Dv + d, s);
-    }
-    // points: aggregate in global frame, back into the query frame
-    for (int qq = lane; qq < Q; qq += 32) {
-      float G[3];
-#pragma unroll
-      for (int x = 0; x < 3; ++x) G[x] = orow[gofs + 3 * qq + x] + orow[gofs + p.Q38 + 3 * qq + x];
-      G[0] += Wv.x - t[0];
-      G[1] += Wv.y - t[1];
-      G[2] += Wv.z - t[2];
-      float L[3];
-#pragma unroll
-      for (int x = 0; x < 3; ++x) L[x] = R[0 * 3 + x] * G[0] + R[1 * 3 + x] * G[1] + R[2 * 3 + x] * G[2];
-      const float len = sqrtf(L[0] * L[0] + L[1] * L[1] + L[2] * L[2] + a.eps);
-      const int base = H * Dv + h * Q + qq;
-      put_feature(frow, F, p.f32, base, L[0]);
-      put_feature(frow, F, p.f32, base + H * Q, L[1]);
-      put_feature(frow, F, p.f32, base + 2 * H * Q, L[2]);
-      put_feature(frow, F, p.f32, base + 3 * H * Q, len);
-      float* lp = lrow + ((size_t)h * Q + qq) * 3;
-      lp[0] = L[0]; lp[1] = L[1]; lp[2] = L[2];
-    }
-    // pair block through the factors
-    for (int c = lane; c < Cz; c += 32) {
-      float acc = 0.f;
-      for (int r = 0; r < p.R; ++r) {
-        float u = orow[p.VHp + r * Cz + c];
-        if (p.f32) u += orow[p.VHp + p.RC8 + r * Cz + c];
-        acc = fmaf(ld_in(z1, bi * RCz + r * Cz + c), u, acc);
-      }
-      put_feature(frow, F, p.f32, H * Dv + 4 * H * Q + h * Cz + c, acc);
-    }
-  }
-}
-
 // w_out [F, Cout] -> wT [Cout_pad, Kgp] fp16, K-major, matching the feature parts:
 //   bf16 inputs: [ w | w ]            (w is exact in fp16)
 //   f32  inputs: [ w hi | w lo | w hi ]
+// 32 x 32 tiles transposed through shared memory (coalesced reads and writes).
 template <typename T>
-__global__ void fipa_weight_prep_kernel(const Plan p, const T* w, __half* wT, int cout_pad) {
-  const size_t n_el = (size_t)cout_pad * p.Kgp;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < n_el; e += (size_t)gridDim.x * blockDim.x) {
-    const int n = (int)(e / p.Kgp), kk = (int)(e % p.Kgp);
-    float v = 0.f;
-    int is_lo = 0;
-    if (n < p.Cout && kk < p.Kg) {
-      const int seg = kk / p.F, f = kk - seg * p.F;
-      v = ld_in(w, (size_t)f * p.Cout + n);
-      is_lo = (p.f32 && seg == 1);
+__global__ void __launch_bounds__(256) fipa_weight_prep_kernel(const Plan p, const T* w, __half* wT, int cout_pad) {
+  __shared__ float tile[32][33];
+  const int f0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int k = ty; k < 32; k += 8) {
+    const int f = f0 + k, n = n0 + tx;
+    tile[k][tx] = (f < p.F && n < p.Cout) ? ld_in(w, (size_t)f * p.Cout + n) : 0.f;
+  }
+  __syncthreads();
+  const int nseg = p.f32 ? 3 : 2;
+  for (int k = ty; k < 32; k += 8) {
+    const int n = n0 + k, f = f0 + tx;
+    if (n >= cout_pad || f >= p.F) continue;
+    const float v = tile[tx][k];
+    const __half hi = __float2half_rn(v), lo = __float2half_rn(v - __half2float(hi));
+    for (int seg = 0; seg < nseg; ++seg) wT[(size_t)n * p.Kgp + seg * p.F + f] = (p.f32 && seg == 1) ? lo : hi;
+  }
+  if (blockIdx.x == 0) {
+    for (int k = ty; k < 32; k += 8) {
+      const int n = n0 + k;
+      if (n < cout_pad)
+        for (int c = p.Kg + tx; c < p.Kgp; c += 32) wT[(size_t)n * p.Kgp + c] = __float2half_rn(0.f);
     }
-    const __half hi = __float2half_rn(v);
-    wT[e] = is_lo ? __float2half_rn(v - __half2float(hi)) : hi;
+  }
+}
+
+// Sum of the split-K partials, + b_out, zero for an empty neighbourhood.
+template <typename T>
+__global__ void fipa_proj_reduce_kernel(const Plan p, const float* part, const T* b_out, const uint8_t* rowflag,
+                                        float* update) {
+  const int cpad = rup(p.Cout, p.ntile_out);
+  const size_t total = (size_t)p.B * p.N * p.Cout, plane = (size_t)p.B * p.N * cpad;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = e / p.Cout;
+    const int n = (int)(e - m * p.Cout);
+    float acc = 0.f;
+    for (int z = 0; z < p.gemm_ks; ++z) acc += part[z * plane + m * cpad + n];
+    update[e] = rowflag[m] ? acc + ld_in(b_out, n) : 0.f;
   }
 }
 
@@ -132,6 +65,7 @@ struct ProjArgs {
   const void* b_out;
   const uint8_t* rowflag;
   float* update;
+  float* part;
   int* status;
   unsigned long long timeout_ns;
 };
@@ -156,7 +90,9 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   int* abort_flag = reinterpret_cast<int*>(tail + 260);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kTile, n0 = blockIdx.y * ntile;
-  const int nk = p.Kgp / kChunk;
+  const int nk_all = p.Kgp / kChunk;
+  const int k0 = blockIdx.z * p.gemm_nks;
+  const int nk = min(nk_all, k0 + p.gemm_nks) - k0;      // K chunks of this split
   const uint32_t ncols = ntile <= 32 ? 32 : ntile <= 64 ? 64 : ntile <= 128 ? 128 : 256;
 
   if (threadIdx.x == 0) {
@@ -182,8 +118,8 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         if (!mbar_wait(&empty[st], ph ^ 1u, wc, 21)) break;
         uint8_t* sa = smem + (size_t)st * stage;
         mbar_arrive_expect_tx(&full[st], (uint32_t)stage);
-        tma_load_2d(sa, &tmA, &full[st], c * kChunk, m0);
-        tma_load_2d(sa + kChunkBytes, &tmB, &full[st], c * kChunk, n0);
+        tma_load_2d(sa, &tmA, &full[st], (k0 + c) * kChunk, m0);
+        tma_load_2d(sa + kChunkBytes, &tmB, &full[st], (k0 + c) * kChunk, n0);
         ++issued;
         if (++st == nst) { st = 0; ph ^= 1u; }
       }
@@ -227,11 +163,16 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const bool live = m < p.B * p.N;
       const bool keep = live && a.rowflag[m] != 0;
       const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
+      const int cpad = rup(p.Cout, ntile);
+      float* prow = a.part + ((size_t)blockIdx.z * p.B * p.N + (size_t)m) * cpad;
       for (int c = 0; c < ntile; c += 32) {
         uint32_t o[32];
         tmem_ld32(trow + (uint32_t)c, o);
         tmem_ld_wait();
-        if (live) {
+        if (live && p.gemm_ks > 1) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) prow[n0 + c + e] = __uint_as_float(o[e]);
+        } else if (live) {
           float* urow = a.update + (size_t)m * p.Cout;
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -257,34 +198,37 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
 }  // namespace
 
-cudaError_t launch_features(const Plan& p, const Inputs& in, const Work& w, const Outputs& out, cudaStream_t s) {
-  FeatArgs a{p, in.rot, in.trans, in.z1, w.O, w.W, w.feat, w.rowflag, out.local_points, in.eps};
-  const size_t BN = (size_t)p.B * p.N;
-  const unsigned grid = (unsigned)((BN + kFeatWarps - 1) / kFeatWarps);
-  if (p.f32) fipa_features_kernel<float><<<grid, kFeatWarps * 32, 0, s>>>(a);
-  else fipa_features_kernel<__nv_bfloat16><<<grid, kFeatWarps * 32, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_weight_prep(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s) {
   const int cout_pad = rup(p.Cout, p.ntile_out);
-  const size_t n_el = (size_t)cout_pad * p.Kgp;
-  unsigned grid = (unsigned)((n_el + 255) / 256);
-  if (grid > 4096) grid = 4096;
-  if (p.f32) fipa_weight_prep_kernel<float><<<grid, 256, 0, s>>>(p, static_cast<const float*>(in.w_out), w.wT, cout_pad);
-  else fipa_weight_prep_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p, static_cast<const __nv_bfloat16*>(in.w_out), w.wT, cout_pad);
+  dim3 grid((unsigned)cdiv(p.F, 32), (unsigned)cdiv(cout_pad, 32)), block(32, 8);
+  if (p.f32)
+    fipa_weight_prep_kernel<float><<<grid, block, 0, s>>>(p, static_cast<const float*>(in.w_out), w.wT, cout_pad);
+  else
+    fipa_weight_prep_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
+        p, static_cast<const __nv_bfloat16*>(in.w_out), w.wT, cout_pad);
   return cudaGetLastError();
 }
 
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl, cudaStream_t s) {
-  ProjArgs a{p, in.b_out, w.rowflag, out.update, ctl.status, ctl.timeout_ns};
+  ProjArgs a{p, in.b_out, w.rowflag, out.update, w.part, ctl.status, ctl.timeout_ns};
   const size_t BN = (size_t)p.B * p.N;
-  dim3 grid((unsigned)((BN + kTile - 1) / kTile), (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out));
-  cudaError_t e = cudaFuncSetAttribute(fipa_out_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)p.gemm_smem);
+  dim3 grid((unsigned)((BN + kTile - 1) / kTile), (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out),
+            (unsigned)p.gemm_ks);
+  cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_out_proj_kernel));
   if (e != cudaSuccess) return e;
   fipa_out_proj_kernel<<<grid, 256, p.gemm_smem, s>>>(tmA, tmB, a);
+  if (p.gemm_ks > 1) {
+    const size_t total = BN * p.Cout;
+    unsigned g = (unsigned)((total + 255) / 256);
+    if (g > 148 * 16) g = 148 * 16;
+    if (p.f32)
+      fipa_proj_reduce_kernel<float><<<g, 256, 0, s>>>(p, w.part, static_cast<const float*>(in.b_out), w.rowflag,
+                                                         out.update);
+    else
+      fipa_proj_reduce_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
+          p, w.part, static_cast<const __nv_bfloat16*>(in.b_out), w.rowflag, out.update);
+  }
   return cudaGetLastError();
 }
 

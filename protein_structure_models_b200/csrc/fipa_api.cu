@@ -29,7 +29,10 @@ struct fipa_handle {
   std::string last_error;
   bool timing = false;
   bool timed_call = false;
-  cudaEvent_t ev[7] = {};
+  cudaEvent_t ev[6] = {};
+  long long* d_trace = nullptr;
+  int trace_cta = -1;
+  int pair_split = 1;
 };
 
 namespace {
@@ -76,7 +79,7 @@ fipa_status encode_rows(fipa_handle* h, CUtensorMap* m, const void* base, uint64
 int plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
   const char* why = "";
   int rc = fipa::make_plan(p, d->B, d->N, d->H, d->D, d->Dv, d->P, d->Q, d->Cz, d->R, d->Cout,
-                           h->dtype == FIPA_F32 ? 1 : 0, &why);
+                           h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split);
   if (rc != 0) h->last_error = why;
   return rc;
 }
@@ -134,6 +137,12 @@ FIPA_API fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims, f
     return FIPA_ERR_CUDA;
   }
   h->encode = reinterpret_cast<EncodeTiledFn>(fn);
+  if (const char* env = std::getenv("FIPA_PAIR_SPLIT")) h->pair_split = std::strtol(env, nullptr, 10) != 0;
+  if (const char* env = std::getenv("FIPA_TRACE_CTA")) {
+    h->trace_cta = (int)std::strtol(env, nullptr, 10);
+    const size_t bytes = (size_t)4 * FIPA_TRACE_CAP * 2 * sizeof(long long);
+    if (cudaMalloc(&h->d_trace, bytes) != cudaSuccess) { delete h; return FIPA_ERR_CUDA; }
+  }
   if (cudaMalloc(&h->d_status, 256) != cudaSuccess || cudaMemset(h->d_status, 0, 256) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     if (h->d_status) cudaFree(h->d_status);
@@ -165,9 +174,9 @@ FIPA_API fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n) {
   if (h == nullptr || ms == nullptr || n < 0) return FIPA_ERR_INVALID_ARG;
   if (!h->timing || !h->timed_call) return fail(h, FIPA_ERR_INVALID_ARG, "no timed fipa_forward call");
   DeviceGuard g(h->device);
-  cudaError_t e = cudaEventSynchronize(h->ev[6]);
+  cudaError_t e = cudaEventSynchronize(h->ev[5]);
   if (e != cudaSuccess) return cuda_fail(h, "event sync", e);
-  for (int k = 0; k < 6 && k < n; ++k) {
+  for (int k = 0; k < 5 && k < n; ++k) {
     float t = 0.f;
     e = cudaEventElapsedTime(&t, h->ev[k], h->ev[k + 1]);
     if (e != cudaSuccess) return cuda_fail(h, "event time", e);
@@ -181,6 +190,7 @@ FIPA_API fipa_status fipa_destroy(fipa_handle* h) {
   {
     DeviceGuard g(h->device);
     if (h->d_status) cudaFree(h->d_status);
+    if (h->d_trace) cudaFree(h->d_trace);
     if (h->timing)
       for (auto& e : h->ev) cudaEventDestroy(e);
   }
@@ -196,6 +206,31 @@ FIPA_API fipa_status fipa_workspace_size(const fipa_handle* hc, const fipa_dims*
   if (rc == 1) return FIPA_ERR_INVALID_ARG;
   if (rc == 2) return FIPA_ERR_UNSUPPORTED;
   *bytes = p.total;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_trace_copy(fipa_handle* h, int64_t* host, size_t n_values, void* stream) {
+  if (h == nullptr || host == nullptr) return FIPA_ERR_INVALID_ARG;
+  const size_t need = (size_t)4 * FIPA_TRACE_CAP * 2;
+  if (h->d_trace == nullptr || n_values < need) return fail(h, FIPA_ERR_INVALID_ARG, "tracing is off or buffer too small");
+  DeviceGuard g(h->device);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, "stream", e);
+  e = cudaMemcpy(host, h->d_trace, need * sizeof(long long), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, "trace copy", e);
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_kernel_count(const fipa_handle* hc, const fipa_dims* dims, int with_attention,
+                                       int* count) {
+  fipa_handle* h = const_cast<fipa_handle*>(hc);
+  if (h == nullptr || dims == nullptr || count == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "null argument");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  // origin, lift, core, weight prep, projection (+ split-K reduce) (+ attention)
+  *count = 5 + (p.gemm_ks > 1 ? 1 : 0) + (with_attention ? 1 : 0);
   return FIPA_OK;
 }
 
@@ -268,17 +303,17 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   w.qvec = reinterpret_cast<float4*>(ws + p.off_qvec);
   w.orig = reinterpret_cast<float4*>(ws + p.off_orig);
   w.flag = reinterpret_cast<int*>(ws + p.off_flag);
-  w.O = reinterpret_cast<float*>(ws + p.off_O);
-  w.W = reinterpret_cast<float4*>(ws + p.off_W);
   w.stats = reinterpret_cast<float2*>(ws + p.off_stats);
   w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
   w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
   w.rowflag = ws + p.off_rowflag;
+  w.part = reinterpret_cast<float*>(ws + p.off_part);
 
   fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
                   w_out, b_out, (float)eps};
   fipa::Outputs out{out_update, out_local_points, out_attention, out_lse};
-  fipa::DeviceCtl ctl{h->d_status, h->timeout_ns};
+  fipa::DeviceCtl ctl{h->d_status, h->timeout_ns, h->d_trace, h->trace_cta};
+  if (h->d_trace != nullptr) cudaMemsetAsync(h->d_trace, 0xff, (size_t)4 * FIPA_TRACE_CAP * 2 * sizeof(long long), s);
   const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
 
   CUtensorMap tmQ, tmKH, tmVH, tmZ, tmA, tmB;
@@ -294,8 +329,13 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
 
   cudaError_t e;
   const bool rec = h->timing;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (rec) cudaStreamIsCapturing(s, &cap);
+  // inside a stream capture the events become event-record nodes of the graph,
+  // so each replay re-records them and fipa_stage_times reads the replay
+  const unsigned rec_flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
   auto mark = [&](int k) {
-    if (rec) cudaEventRecord(h->ev[k], s);
+    if (rec) cudaEventRecordWithFlags(h->ev[k], s, rec_flags);
   };
   mark(0);
   if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
@@ -305,16 +345,14 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   mark(2);
   if ((e = fipa::launch_weight_prep(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "weight prep launch", e);
   mark(3);
-  if ((e = fipa::launch_features(p, in, w, out, s)) != cudaSuccess) return cuda_fail(h, "features launch", e);
-  mark(4);
   if ((e = fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s)) != cudaSuccess)
     return cuda_fail(h, "output projection launch", e);
-  mark(5);
+  mark(4);
   if (out_attention != nullptr) {
     if ((e = fipa::launch_attention_dump(p, in, w, out, s)) != cudaSuccess)
       return cuda_fail(h, "attention launch", e);
   }
-  mark(6);
+  mark(5);
   h->timed_call = rec;
   return FIPA_OK;
 }

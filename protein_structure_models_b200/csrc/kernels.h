@@ -6,9 +6,36 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "plan.h"
 
 namespace fipa {
+
+// Allow a kernel the full opt-in dynamic shared memory, once per kernel and
+// device: the attribute only bounds the launch-time request, and setting it on
+// every call would cost host time on every forward.
+inline cudaError_t allow_max_smem(const void* kfn) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, bool> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(kfn, dev);
+  if (done.count(key)) return cudaSuccess;
+  int optin = 0;
+  e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kfn);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
+  if (e == cudaSuccess) done[key] = true;
+  return e;
+}
 
 // Inputs exactly as the C ABI receives them (dtype fixed by Plan::f32).
 struct Inputs {
@@ -27,12 +54,11 @@ struct Work {
   float4 *qvec;    // [B*H, N] {sum_p a', -g sum_p |a'|^2}
   float4 *orig;    // [B, nG]  {32-residue group origin xyz, valid residues in group}
   int *flag;       // [B, nT]  tile has a valid residue
-  float *O;        // [B, N, H, Ocols] normalised aggregates of the lifted value columns
-  float4 *W;       // [B, N, H]  {sum_j a_ij o_G(j) (xyz), l}
   float2 *stats;   // [B, H, N]  {running max M (log2 units), softmax denominator l}
   __half *feat;    // [B*N, Kgp] output-projection operand (feature hi/lo halves)
   __half *wT;      // [Cout_pad, Kgp] output-projection weights, K-major
   uint8_t *rowflag;// [B*N] row has a non-empty neighbourhood
+  float *part;     // [gemm_ks, B*N, Cout_pad] split-K partial sums of the projection
 };
 
 struct Outputs {
@@ -42,6 +68,23 @@ struct Outputs {
 struct DeviceCtl {
   int *status;
   unsigned long long timeout_ns;
+  long long *trace;   // debug event log of one core CTA, or null
+  int trace_cta;
+};
+
+constexpr int kTraceCap = 4096;   // events per role of the debug trace (== FIPA_TRACE_CAP)
+
+// Debug event log of one warp role: (event id, SM clock) pairs.
+struct Tracer {
+  long long* buf;
+  int n;
+  __device__ __forceinline__ void ev(int id) {
+    if (buf != nullptr && n < kTraceCap) {
+      buf[2 * n] = id;
+      buf[2 * n + 1] = clock64();
+      ++n;
+    }
+  }
 };
 
 // Launchers return the cudaError_t of the launch.
@@ -49,8 +92,6 @@ cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cuda
 cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                         const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
                         const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s);
-cudaError_t launch_features(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
-                            cudaStream_t s);
 cudaError_t launch_weight_prep(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl,

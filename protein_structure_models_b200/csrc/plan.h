@@ -40,8 +40,14 @@ constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
 constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
 
-static inline int cdiv(int a, int b) { return (a + b - 1) / b; }
-static inline int rup(int a, int b) { return cdiv(a, b) * b; }
+#ifdef __CUDACC__
+#define FIPA_HD __host__ __device__
+#else
+#define FIPA_HD
+#endif
+
+FIPA_HD static inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+FIPA_HD static inline int rup(int a, int b) { return cdiv(a, b) * b; }
 static inline size_t rup_sz(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
 struct Plan {
@@ -69,17 +75,21 @@ struct Plan {
   size_t lift_smem;   // dynamic shared memory of the prologue lift kernel
   int Kg, Kgp;        // output-projection K (2F or 3F) and padded
   int ntile_out;      // output-projection N tile (<= 256)
+  int gemm_ks;        // output-projection split-K factor
+  int gemm_nks;       // K chunks per split
   int gemm_nst;
   size_t gemm_smem;
   // workspace byte offsets
   size_t off_Q, off_KH, off_VH, off_Z, off_kvec, off_qvec, off_orig, off_flag;
   size_t off_QP, off_KP;
-  size_t off_O, off_W, off_stats, off_feat, off_wT, off_rowflag, total;
+  size_t off_stats, off_feat, off_wT, off_rowflag, off_part, total;
 };
 
 // Returns 0 and fills `p`, or a nonzero reason code: 1 = bad dims, 2 = unsupported.
+// pair_split: 1 = pair-bias operand as fp16 hi + lo halves (bfloat16 inputs);
+// 0 = hi half only.
 static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, int Q, int Cz, int R,
-                            int Cout, int f32, const char** why) {
+                            int Cout, int f32, const char** why, int pair_split = 1) {
   *why = "";
   if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || Dv <= 0 || P <= 0 || Q <= 0 || Cz <= 0 || R <= 0 ||
       Cout <= 0) {
@@ -95,7 +105,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.nsv = f32 ? 2 : 1;
   p.nz = f32 ? 3 : 1;
   p.nzv = f32 ? 2 : 1;
-  p.nqz = f32 ? 1 : 2;
+  p.nqz = f32 ? 1 : (pair_split ? 2 : 1);
   p.geo_simt = f32 ? 1 : 0;
   p.D8 = rup(D, 8);
   p.P38 = rup(3 * P, 8);
@@ -136,6 +146,9 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.nst = nst;
   p.core_smem = fixed + (size_t)(p.nQc + nst) * 16384;
   if (p.core_smem < 120 * 1024) p.core_smem = 120 * 1024;   // one CTA per SM (TMEM is taken whole)
+  if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)(p.nQc + nst) * 16384) {
+    *why = "value width too large for the epilogue staging"; return 2;
+  }
   // prologue lift kernel: Wb^T, z1 rows, global points, frames of 8 residues
   p.lift_smem = ((size_t)H * Cz + (size_t)8 * 2 * R * Cz + (size_t)8 * H * (2 * P + Q) * 3 + 8 * 12 +
                  (size_t)8 * H * (2 * D + Dv)) * 4;
@@ -143,11 +156,21 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   // output projection
   p.Kg = (f32 ? 3 : 2) * p.F;
   p.Kgp = rup(p.Kg, kChunk);
-  p.ntile_out = Cout >= 256 ? 256 : rup(Cout, 16);
+  // N tile and split-K so that the grid covers the SMs (deterministic split-K:
+  // partial sums go to the workspace and a reduce kernel adds them in order)
   {
+    const int mt = cdiv(B * N, kTile), nk = p.Kgp / kChunk;
+    int nt_w = Cout >= 256 ? 256 : rup(Cout, 16);
+    while (mt * cdiv(Cout, nt_w) < 148 && nt_w > 64) nt_w = rup(nt_w / 2, 16);
+    p.ntile_out = nt_w;
+    const int tiles = mt * cdiv(Cout, nt_w);
+    int ks = tiles >= 148 ? 1 : cdiv(148, tiles);
+    if (ks > nk / 4) ks = nk / 4 > 1 ? nk / 4 : 1;
+    p.gemm_nks = cdiv(nk, ks);
+    p.gemm_ks = cdiv(nk, p.gemm_nks);
     size_t stage = 16384 + (size_t)p.ntile_out * 128;
     int g = (int)((limit - 2048) / stage);
-    p.gemm_nst = g > 4 ? 4 : g;
+    p.gemm_nst = g > 8 ? 8 : g;
     p.gemm_smem = 2048 + stage * p.gemm_nst;
   }
   // workspace layout
@@ -164,12 +187,11 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.off_qvec = take(BHN * 16);
   p.off_orig = take((size_t)B * p.nG * 16);
   p.off_flag = take((size_t)B * p.nT * 4);
-  p.off_O = take(BN * H * p.Ocols * 4);
-  p.off_W = take(BN * H * 16);
   p.off_stats = take(BHN * 8);
   p.off_feat = take(BN * p.Kgp * 2);
   p.off_wT = take((size_t)rup(Cout, p.ntile_out) * p.Kgp * 2);
   p.off_rowflag = take(BN);
+  p.off_part = take(p.gemm_ks > 1 ? (size_t)p.gemm_ks * BN * rup(Cout, p.ntile_out) * 4 : 0);
   p.total = o;
   return 0;
 }

@@ -182,113 +182,122 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     }
   }
 
-  // ---- every lifted row as 16-byte chunks (8 fp16 values of one segment)
-  const int qc = p.Kq / 8, kc = p.KHp / 8, vc = p.VHp / 8, zc = p.Zp / 8;
-  const int cpr = H * (qc + kc + vc) + zc;          // chunks per residue
+  // ---- every lifted row as 16-byte chunks (8 fp16 values of one segment):
+  // one warp per row, lanes over its chunks
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
   const float sqk = rsqrtf(3.0f * (float)p.D);
-  for (int e = threadIdx.x; e < nres * cpr; e += blockDim.x) {
-    const int r = e / cpr;
-    int c = e - r * cpr;
-    const int i = i0 + r;
-    const size_t bi = (size_t)b * N + i;
+  const int sq = p.nsq * p.D8;          // scalar columns of the query / key head part
+  const int sv = p.nsv * p.Dv8;         // scalar columns of the value head part
+  for (int row = warp; row < nres * H; row += nwarp) {
+    const int r = row / H, h = row - r * H, i = i0 + r;
     const bool valid = s_valid[r] != 0;
-    float vals[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) vals[t] = 0.f;
-    bool lo = false;
-    __half* dst;
-    if (c < H * qc) {                                  // ---- query row of head h
-      const int h = c / qc, col = (c - h * qc) * 8;
-      dst = a.w.Q + (((size_t)b * H + h) * N + i) * p.Kq + col;
+    const float* qsr = qs + (r * H + h) * p.D;
+    const float* ksr = ks + (r * H + h) * p.D;
+    const float* vsr = vs + (r * H + h) * p.Dv;
+    const float* pa = pts + ((size_t)r * H + h) * npt * 3;
+    const float* pb = pa + 3 * P;
+    const float* pg = pb + 3 * P;
+    const float g2 = 2.f * s_gamma[h < 64 ? h : 63];
+    const size_t rowid = ((size_t)b * H + h) * N + i;
+    // query row: [ scalar | points (tensor-core mode) | pad ] [ pair part ]
+    __half* qrow = a.w.Q + rowid * p.Kq;
+    for (int c8 = lane; c8 < p.Kq / 8; c8 += 32) {
+      const int col = c8 * 8;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      bool lo = false;
       if (valid) {
-        if (col < p.KHp) {
-          const int sc = p.nsq * p.D8;
-          if (col < sc) {
-            const int seg = col / p.D8, e0 = col - seg * p.D8;
+        if (col < sq) {
+          const int seg = col / p.D8, e0 = col - seg * p.D8;
+          lo = (seg == 2);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) if (e0 + t < p.D) v[t] = qsr[e0 + t] * sqk;
+        } else if (col < p.KHp) {
+          if (!p.geo_simt && col < sq + 3 * p.P38) {
+            const int seg = (col - sq) / p.P38, e0 = col - sq - seg * p.P38;
             lo = (seg == 2);
 #pragma unroll
-            for (int t = 0; t < 8; ++t)
-              if (e0 + t < p.D) vals[t] = qs[(r * H + h) * p.D + e0 + t] * sqk;
-          } else if (!p.geo_simt && col < sc + 3 * p.P38) {
-            const int seg = (col - sc) / p.P38, e0 = col - sc - seg * p.P38;
-            const float g2 = 2.f * s_gamma[h < 64 ? h : 63];
-            const float* pa = pts + ((size_t)r * H + h) * npt * 3;
-            lo = (seg == 2);
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              if (e0 + t < 3 * P) vals[t] = g2 * pa[e0 + t];
+            for (int t = 0; t < 8; ++t) if (e0 + t < 3 * P) v[t] = g2 * pa[e0 + t];
           }
         } else {
-          int cc = col - p.KHp, e0;
-          if (p.nqz == 2) {                          // [u hi | u lo], each Zp wide
+          const int cc = col - p.KHp;
+          int e0;
+          if (p.nqz == 2) {                        // [u hi | u lo], each Zp wide
             lo = cc >= p.Zp;
             e0 = lo ? cc - p.Zp : cc;
-          } else {                                   // [u hi | u hi | u lo], RC8 apart
+          } else {                                 // [u hi | u hi | u lo], RC8 apart
             const int seg = cc / p.RC8;
             e0 = seg < p.nz ? cc - seg * p.RC8 : RCz;
             lo = (seg == 2);
           }
-          int rr = e0 / Cz, c0 = e0 - rr * Cz;
+          if (e0 < RCz) {
+            int rr = e0 / Cz, c0 = e0 - rr * Cz;
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            if (e0 + t < RCz) vals[t] = z1s[r * RCz + e0 + t] * wbt[h * Cz + c0];
-            if (++c0 == Cz) { c0 = 0; ++rr; }
+            for (int t = 0; t < 8; ++t) {
+              if (e0 + t < RCz) v[t] = z1s[r * RCz + e0 + t] * wbt[h * Cz + c0];
+              if (++c0 == Cz) { c0 = 0; ++rr; }
+            }
           }
         }
       }
-    } else if ((c -= H * qc) < H * kc) {               // ---- key row (head part)
-      const int h = c / kc, col = (c - h * kc) * 8;
-      dst = a.w.KH + (((size_t)b * H + h) * N + i) * p.KHp + col;
-      const int sc = p.nsq * p.D8;
+      store8(qrow + col, v, lo);
+    }
+    // key row (head part): [ scalar | points (tensor-core mode) | pad ]
+    __half* krow = a.w.KH + rowid * p.KHp;
+    for (int c8 = lane; c8 < p.KHp / 8; c8 += 32) {
+      const int col = c8 * 8;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      bool lo = false;
       if (valid) {
-        if (col < sc) {
+        if (col < sq) {
           const int seg = col / p.D8, e0 = col - seg * p.D8;
           lo = (seg == 1);
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (e0 + t < p.D) vals[t] = ks[(r * H + h) * p.D + e0 + t];
-        } else if (!p.geo_simt && col < sc + 3 * p.P38) {
-          const int seg = (col - sc) / p.P38, e0 = col - sc - seg * p.P38;
-          const float* pb = pts + ((size_t)r * H + h) * npt * 3 + 3 * P;
+          for (int t = 0; t < 8; ++t) if (e0 + t < p.D) v[t] = ksr[e0 + t];
+        } else if (!p.geo_simt && col < sq + 3 * p.P38) {
+          const int seg = (col - sq) / p.P38, e0 = col - sq - seg * p.P38;
           lo = (seg == 1);
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (e0 + t < 3 * P) vals[t] = pb[e0 + t];
+          for (int t = 0; t < 8; ++t) if (e0 + t < 3 * P) v[t] = pb[e0 + t];
         }
       }
-    } else if ((c -= H * kc) < H * vc) {               // ---- value row (head part)
-      const int h = c / vc, col = (c - h * vc) * 8;
-      dst = a.w.VH + (((size_t)b * H + h) * N + i) * p.VHp + col;
-      const int sc = p.nsv * p.Dv8;
+      store8(krow + col, v, lo);
+    }
+    // value row (head part): [ scalar | g' hi | g' lo | pad ]
+    __half* vrow = a.w.VH + rowid * p.VHp;
+    for (int c8 = lane; c8 < p.VHp / 8; c8 += 32) {
+      const int col = c8 * 8;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      bool lo = false;
       if (valid) {
-        if (col < sc) {
+        if (col < sv) {
           const int seg = col / p.Dv8, e0 = col - seg * p.Dv8;
           lo = (seg == 1);
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (e0 + t < p.Dv) vals[t] = vs[(r * H + h) * p.Dv + e0 + t];
-        } else if (col < sc + 2 * p.Q38) {
-          const int seg = (col - sc) / p.Q38, e0 = col - sc - seg * p.Q38;
-          const float* pg = pts + ((size_t)r * H + h) * npt * 3 + 6 * P;
+          for (int t = 0; t < 8; ++t) if (e0 + t < p.Dv) v[t] = vsr[e0 + t];
+        } else if (col < sv + 2 * p.Q38) {
+          const int seg = (col - sv) / p.Q38, e0 = col - sv - seg * p.Q38;
           lo = (seg == 1);
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            if (e0 + t < 3 * Q) vals[t] = pg[e0 + t];
+          for (int t = 0; t < 8; ++t) if (e0 + t < 3 * Q) v[t] = pg[e0 + t];
         }
       }
-    } else {                                           // ---- pair factor row z2 (shared by heads)
-      c -= H * vc;
-      const int col = c * 8;
-      dst = a.w.Z + bi * p.Zp + col;
-      const int seg = col / p.RC8, e0 = col - seg * p.RC8;
-      if (valid && seg < p.nz) {
-        lo = (seg == 1);
-#pragma unroll
-        for (int t = 0; t < 8; ++t)
-          if (e0 + t < RCz) vals[t] = z2s[r * RCz + e0 + t];
-      }
+      store8(vrow + col, v, lo);
     }
-    store8(dst, vals, lo);
+  }
+  // pair factor rows z2 (shared by the heads): [ z2 segments | pad ]
+  for (int r = warp; r < nres; r += nwarp) {
+    const bool valid = s_valid[r] != 0;
+    __half* zrow = a.w.Z + (bi0 + r) * p.Zp;
+    for (int c8 = lane; c8 < p.Zp / 8; c8 += 32) {
+      const int col = c8 * 8, seg = col / p.RC8, e0 = col - seg * p.RC8;
+      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const bool lo = (seg == 1);
+      if (valid && seg < p.nz) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) if (e0 + t < RCz) v[t] = z2s[r * RCz + e0 + t];
+      }
+      store8(zrow + col, v, lo);
+    }
   }
 }
 
@@ -300,13 +309,13 @@ cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cuda
   if (p.f32) {
     fipa_origin_kernel<float><<<g1, kTile, 0, s>>>(a);
     auto kfn = fipa_lift_kernel<float>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.lift_smem);
+    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
     if (e != cudaSuccess) return e;
     kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
   } else {
     fipa_origin_kernel<__nv_bfloat16><<<g1, kTile, 0, s>>>(a);
     auto kfn = fipa_lift_kernel<__nv_bfloat16>;
-    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.lift_smem);
+    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
     if (e != cudaSuccess) return e;
     kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
   }

@@ -68,6 +68,10 @@ def load_library():
     lib.fipa_enable_stage_timing.restype = c_int
     lib.fipa_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), c_int]
     lib.fipa_stage_times.restype = c_int
+    lib.fipa_trace_copy.argtypes = [vp, ctypes.POINTER(ctypes.c_int64), sz, vp]
+    lib.fipa_trace_copy.restype = c_int
+    lib.fipa_kernel_count.argtypes = [vp, ctypes.POINTER(FipaDims), c_int, ctypes.POINTER(c_int)]
+    lib.fipa_kernel_count.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -123,6 +127,25 @@ class Fipa:
         self._check(self.lib.fipa_workspace_size(self.handle, ctypes.byref(d), ctypes.byref(n)))
         return int(n.value)
 
+    TRACE_CAP = 4096
+
+    def trace(self, stream: Optional[torch.cuda.Stream] = None):
+        """Debug event log of the traced core CTA (needs FIPA_TRACE_CTA at creation):
+        int64 array [4 roles, TRACE_CAP, 2] of (event id, SM clock), -1 = unused."""
+        import numpy as np
+        s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))
+        buf = np.empty((4, self.TRACE_CAP, 2), dtype=np.int64)
+        self._check(self.lib.fipa_trace_copy(self.handle, buf.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                             buf.size, ctypes.c_void_p(s.cuda_stream)))
+        return buf
+
+    def kernel_count(self, dims: dict, with_attention: bool = False) -> int:
+        d = make_dims(**dims)
+        n = ctypes.c_int()
+        self._check(self.lib.fipa_kernel_count(self.handle, ctypes.byref(d), 1 if with_attention else 0,
+                                               ctypes.byref(n)))
+        return int(n.value)
+
     def dims_of(self, inp: dict) -> dict:
         B, N, H, D = inp["q"].shape
         return dict(B=B, N=N, H=H, D=D, Dv=inp["v"].shape[-1], P=inp["q_points"].shape[3],
@@ -166,15 +189,15 @@ class Fipa:
         self._check(st)
         return out
 
-    STAGES = ("prologue", "core", "weight_prep", "features", "out_proj", "attention")
+    STAGES = ("prologue", "core", "weight_prep", "out_proj", "attention")
 
     def enable_stage_timing(self, enable: bool = True):
         self._check(self.lib.fipa_enable_stage_timing(self.handle, 1 if enable else 0))
 
     def stage_times(self) -> dict:
         """Device ms of each stage of the most recent timed forward."""
-        buf = (ctypes.c_float * 6)()
-        self._check(self.lib.fipa_stage_times(self.handle, buf, 6))
+        buf = (ctypes.c_float * 5)()
+        self._check(self.lib.fipa_stage_times(self.handle, buf, 5))
         return dict(zip(self.STAGES, [float(x) for x in buf]))
 
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
