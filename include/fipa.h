@@ -125,6 +125,46 @@ fipa_status fipa_forward(fipa_handle* h,
                          void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/* Allocation-free forward.  No counterpart on the method's pages: this entry
+ * point exists for callers that cannot allocate device memory where they call
+ * the forward, e.g. code running while a CUDA graph is being captured (a
+ * cudaMalloc there is forbidden or breaks the capture) or a plugin whose host
+ * framework owns every device allocation through its own pool.  Such callers
+ * can create neither a workspace nor a handle (fipa_create allocates the
+ * handle's status word), so this call takes neither.
+ *
+ * Scratch: one fixed device array of FIPA_NOALLOC_SCRATCH_BYTES inside the
+ * library, held by every GPU that loads the library until the process exits.
+ * Problems whose fipa_workspace_size exceeds it are rejected with
+ * FIPA_ERR_WORKSPACE before anything is launched.  The call makes no
+ * cudaMalloc / cudaFree and calls no allocating routine.
+ *
+ * Set-up: the first call on each device (the current device at call time)
+ * looks up the array's device address with cudaGetSymbolAddress; make that
+ * first call before any stream capture.
+ *
+ * Sharing: every call uses the same array and leaves its contents behind, so
+ * calls whose kernels could overlap on the GPU (different streams without
+ * ordering between them) race; order them on one stream or with events.
+ * Nothing in the array needs clearing between calls.
+ *
+ * Arguments and outputs are those of fipa_forward (no attention output); the
+ * kernels run asynchronously on `stream`.  A bounded device-side wait that
+ * expires (which only a faulty device or build can cause) leaves the outputs
+ * undefined and is not reported by this call. */
+#define FIPA_NOALLOC_SCRATCH_BYTES (32u << 20)
+fipa_status fipa_forward_noalloc(fipa_dtype dtype,
+                                 const void* q, const void* k, const void* v,
+                                 const void* q_pts, const void* k_pts, const void* v_pts,
+                                 const void* rot, const void* trans,
+                                 const void* z1, const void* z2, const void* Wb,
+                                 const void* point_w_raw,
+                                 const uint8_t* mask, const uint8_t* pair_mask,
+                                 const void* w_out, const void* b_out, double eps,
+                                 const fipa_dims* dims,
+                                 float* out_update, float* out_local_points, float* out_lse,
+                                 void* stream);
+
 /* Wait for `stream`, then read and clear the handle's device status word.
  * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */

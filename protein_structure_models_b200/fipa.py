@@ -72,6 +72,10 @@ def load_library():
     lib.fipa_trace_copy.restype = c_int
     lib.fipa_kernel_count.argtypes = [vp, ctypes.POINTER(FipaDims), c_int, ctypes.POINTER(c_int)]
     lib.fipa_kernel_count.restype = c_int
+    lib.fipa_forward_noalloc.argtypes = [c_int] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double,
+                                                                         ctypes.POINTER(FipaDims)] \
+        + [vp] * 3 + [vp]
+    lib.fipa_forward_noalloc.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -203,6 +207,39 @@ class Fipa:
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))
         self._check(self.lib.fipa_sync_status(self.handle, ctypes.c_void_p(s.cuda_stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def forward_noalloc(inp: dict, eps: float = 1e-8, out: Optional[dict] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """fipa_forward_noalloc: the forward without a handle or a workspace, for
+    callers that may not allocate device memory where they run it (inside a
+    CUDA graph capture, or under a host framework that owns all device
+    allocations).  Its scratch is a fixed 32 MiB device array inside the
+    library; `out`, if given, must hold preallocated "update" and
+    "local_points" (and optionally "lse") tensors, so this path allocates
+    nothing either."""
+    lib = load_library()
+    q = inp["q"]
+    dtype = BF16 if q.dtype == torch.bfloat16 else F32
+    B, N, H, D = q.shape
+    dims = dict(B=B, N=N, H=H, D=D, Dv=inp["v"].shape[-1], P=inp["q_points"].shape[3],
+                Q=inp["v_points"].shape[3], Cz=inp["z1"].shape[3], R=inp["z1"].shape[2],
+                Cout=inp["w_out"].shape[1])
+    if out is None:
+        out = {"update": torch.empty((B, N, dims["Cout"]), dtype=torch.float32, device=q.device),
+               "local_points": torch.empty((B, N, H, dims["Q"], 3), dtype=torch.float32, device=q.device)}
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    d = make_dims(**dims)
+    st = lib.fipa_forward_noalloc(
+        dtype, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]), _ptr(inp.get("pair_mask")),
+        _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d),
+        _ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("lse")), ctypes.c_void_p(s.cuda_stream))
+    if st != FIPA_OK:
+        raise FipaError(st, "fipa_forward_noalloc failed")
+    return out
 
 
 _handles: dict = {}
