@@ -60,20 +60,35 @@ struct WaitCtx {
   uint64_t timeout_ns;
 };
 
+// try_wait that lets the warp sleep until the phase completes (the hardware
+// wakes it) or `hint_ns` passes, instead of spinning on the issue slots that
+// the warps on the critical path share.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for phase `parity` of `bar`.  Returns false (and the caller must wind
-// down) when the budget ran out or another thread of the CTA gave up.
+// down) when the budget ran out or another thread of the CTA gave up.  Each
+// try sleeps at most 0.2 ms, so the budget and the abort flag are re-checked
+// at least that often.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtx& w, int site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
-      if (*w.abort) return false;
-      if (global_timer_ns() - t0 > w.timeout_ns) {
-        *w.abort = 1;
-        atomicCAS(w.status, 0, kDeviceTimeout | (site << 8));
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 200000u)) return true;
+    if (*w.abort) return false;
+    if (global_timer_ns() - t0 > w.timeout_ns) {
+      *w.abort = 1;
+      atomicCAS(w.status, 0, kDeviceTimeout | (site << 8));
+      return false;
     }
   }
 }
