@@ -39,6 +39,7 @@ constexpr int kMaxPts = 64;      // points per head handled by the prologue scra
 constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
 constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
+constexpr int kLiftRes = 8;      // residues per prologue lift CTA (divides the 128-residue tile)
 
 #ifdef __CUDACC__
 #define FIPA_HD __host__ __device__
@@ -47,6 +48,23 @@ constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance)
 #endif
 
 FIPA_HD static inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// Division by an invariant divisor d >= 1 as one wide multiply and a shift
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994): with l = ceil(log2 d), p = 31 + l and
+// m = ceil(2^p / d) (< 2^32), floor(n / d) = floor(n * m / 2^p) for every
+// 0 <= n < 2^31, because m = (2^p + e) / d with 0 <= e < d adds less than
+// n e / (d 2^p) < 2^-l <= 1/d to n / d, which never reaches the next integer.
+struct FastDiv {
+  uint32_t d, m, p;
+  FIPA_HD uint32_t div(uint32_t n) const { return (uint32_t)(((uint64_t)n * m) >> p); }
+};
+static inline FastDiv make_fastdiv(uint32_t d) {
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  const uint32_t p = 31 + l;
+  return FastDiv{d, (uint32_t)(((1ull << p) + d - 1) / d), p};
+}
 FIPA_HD static inline int rup(int a, int b) { return cdiv(a, b) * b; }
 static inline size_t rup_sz(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
@@ -73,6 +91,9 @@ struct Plan {
   int nst;            // shared-memory ring stages of the core kernel
   size_t core_smem;   // dynamic shared memory of the core kernel
   size_t lift_smem;   // dynamic shared memory of the prologue lift kernel
+  FastDiv fd_H, fd_P, fd_Q, fd_Cz;               // divisors of the lift kernel's index maps
+  FastDiv fd_nQ8, fd_nK8, fd_nV8, fd_nZ8;        // 16-byte chunks per lifted row type
+  FastDiv fd_D8v, fd_Dv8v, fd_RC8v;              // 8-value vectors per staged row
   int Kg, Kgp;        // output-projection K (2F or 3F) and padded
   int ntile_out;      // output-projection N tile (<= 256)
   int gemm_ks;        // output-projection split-K factor
@@ -149,9 +170,15 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)(p.nQc + nst) * 16384) {
     *why = "value width too large for the epilogue staging"; return 2;
   }
-  // prologue lift kernel: Wb^T, z1 rows, global points, frames of 8 residues
-  p.lift_smem = ((size_t)H * Cz + (size_t)8 * 2 * R * Cz + (size_t)8 * H * (2 * P + Q) * 3 + 8 * 12 +
-                 (size_t)8 * H * (2 * D + Dv)) * 4;
+  // prologue lift kernel: Wb^T, zero-padded z1 / z2 / q / k / v / point rows
+  // and frames of kLiftRes residues, and the chunk table of the four row types
+  p.lift_smem = ((size_t)rup(H * Cz, 8) + (size_t)kLiftRes * 2 * p.RC8 +
+                 (size_t)kLiftRes * H * (2 * p.D8 + p.Dv8 + 2 * p.P38 + p.Q38) + kLiftRes * 12) * 4 +
+                (size_t)(p.Kq + p.KHp + p.VHp + p.Zp) / 8 * 4;
+  p.fd_H = make_fastdiv(H); p.fd_P = make_fastdiv(P); p.fd_Q = make_fastdiv(Q); p.fd_Cz = make_fastdiv(Cz);
+  p.fd_nQ8 = make_fastdiv(p.Kq / 8); p.fd_nK8 = make_fastdiv(p.KHp / 8);
+  p.fd_nV8 = make_fastdiv(p.VHp / 8); p.fd_nZ8 = make_fastdiv(p.Zp / 8);
+  p.fd_D8v = make_fastdiv(p.D8 / 8); p.fd_Dv8v = make_fastdiv(p.Dv8 / 8); p.fd_RC8v = make_fastdiv(p.RC8 / 8);
   if (p.lift_smem > 160 * 1024) { *why = "prologue staging exceeds shared memory (H*Cz or R*Cz too large)"; return 2; }
   // output projection
   p.Kg = (f32 ? 3 : 2) * p.F;

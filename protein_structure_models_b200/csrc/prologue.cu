@@ -19,7 +19,6 @@
 namespace fipa {
 namespace {
 
-constexpr int kLiftRes = 8;        // residues per lift CTA (divides the 128-residue tile)
 constexpr int kLiftThreads = 256;
 
 __device__ __forceinline__ __half hi_half(float x) { return __float2half_rn(x); }
@@ -73,57 +72,213 @@ __global__ void __launch_bounds__(kTile) fipa_origin_kernel(const PrologueArgs a
   if (threadIdx.x == 0) a.w.flag[(size_t)b * p.nT + t] = (s_any[0] | s_any[1] | s_any[2] | s_any[3]) ? 1 : 0;
 }
 
+
+// ---- lift: chunk descriptors
+// Every 16-byte chunk (8 fp16 columns) of a lifted row reads 8 consecutive
+// fp32 values of one zero-padded source row in shared memory.  A per-CTA table
+// holds, for each chunk position of each row type, which source it reads, at
+// which offset, and whether it stores the hi or the lo half; the write loop
+// then does no index arithmetic beyond one table load per chunk.
+enum : uint32_t { kSrcZero = 0, kSrcScalar = 1, kSrcPoint = 2, kSrcPair = 3, kSrcZ2 = 4 };
+enum : int { kRowQ = 0, kRowK = 1, kRowV = 2, kRowZ = 3 };
+
+__device__ __forceinline__ uint32_t make_desc(uint32_t src, int off, int woff, bool lo) {
+  return (uint32_t)off | ((uint32_t)woff << 11) | (src << 22) | ((lo ? 1u : 0u) << 26);
+}
+
+// Descriptor of the chunk starting at column `col` of a row of type `rt`,
+// following the column layout of plan.h.  Point offsets index the per-(residue,
+// head) point row [a' (P38) | b' (P38) | g' (Q38)].
+__device__ uint32_t chunk_desc(const Plan& p, int rt, int col) {
+  const int RCz = p.R * p.Cz;
+  if (rt == kRowZ) {
+    const int seg = col / p.RC8, e0 = col - seg * p.RC8;
+    return seg < p.nz ? make_desc(kSrcZ2, e0, 0, seg == 1) : make_desc(kSrcZero, 0, 0, false);
+  }
+  if (rt == kRowV) {
+    const int sv = p.nsv * p.Dv8;
+    if (col < sv) {
+      const int seg = col / p.Dv8;
+      return make_desc(kSrcScalar, col - seg * p.Dv8, 0, seg == 1);
+    }
+    if (col < sv + 2 * p.Q38) {
+      const int seg = (col - sv) / p.Q38;
+      return make_desc(kSrcPoint, 2 * p.P38 + (col - sv - seg * p.Q38), 0, seg == 1);
+    }
+    return make_desc(kSrcZero, 0, 0, false);
+  }
+  // query (rt 0) and key (rt 1) head parts: the lo copy is segment 2 on the
+  // query side and segment 1 on the key side
+  const int lo_seg = rt == kRowQ ? 2 : 1;
+  const int sq = p.nsq * p.D8;
+  if (col < sq) {
+    const int seg = col / p.D8;
+    return make_desc(kSrcScalar, col - seg * p.D8, 0, seg == lo_seg);
+  }
+  if (col < p.KHp) {
+    if (!p.geo_simt && col < sq + 3 * p.P38) {
+      const int seg = (col - sq) / p.P38;
+      return make_desc(kSrcPoint, (rt == kRowQ ? 0 : p.P38) + (col - sq - seg * p.P38), 0, seg == lo_seg);
+    }
+    return make_desc(kSrcZero, 0, 0, false);
+  }
+  // query pair part: u = z1[r,c] Wb[c,h] / sqrt(3)
+  const int cc = col - p.KHp;
+  int e0;
+  bool lo;
+  if (p.nqz == 2) {                       // [u hi | u lo], each Zp wide
+    lo = cc >= p.Zp;
+    e0 = lo ? cc - p.Zp : cc;
+  } else {                                // [u hi | u hi | u lo], RC8 apart
+    const int seg = cc / p.RC8;
+    e0 = seg < p.nz ? cc - seg * p.RC8 : RCz;
+    lo = (seg == 2);
+  }
+  if (e0 >= RCz) return make_desc(kSrcZero, 0, 0, false);
+  const int rr = e0 / p.Cz;
+  return make_desc(kSrcPair, e0, e0 - rr * p.Cz, lo);
+}
+
+__device__ __forceinline__ void lds8(const float* src, float (&v)[8]) {
+  const float4 a = reinterpret_cast<const float4*>(src)[0], b = reinterpret_cast<const float4*>(src)[1];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void sts8(float* dst, const float (&v)[8]) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+// Round 8 values to fp16 (hi), or store the rounding residual x - fp16(x) (lo).
+__device__ __forceinline__ void stg8_half(__half* dst, const float (&v)[8], bool lo) {
+  uint32_t w[4];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const __half2 h = __floats2half2_rn(v[2 * t], v[2 * t + 1]);
+    if (lo) {
+      const float2 f = __half22float2(h);
+      w[t] = h2_bits(__floats2half2_rn(v[2 * t] - f.x, v[2 * t + 1] - f.y));
+    } else {
+      w[t] = h2_bits(h);
+    }
+  }
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 8 consecutive inputs as fp32 (16-byte aligned source: one or two vector loads).
+__device__ __forceinline__ void ldg8(const float* src, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src)), b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ldg8(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    v[2 * t] = __uint_as_float(w[t] << 16);
+    v[2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
+  }
+}
+
+// Stage `nrows` contiguous input rows of L values into shared rows of L8
+// (a multiple of 8; fd_vec divides by L8 / 8) floats, times `scale`, zero-padded.
+template <typename T>
+__device__ __forceinline__ void stage_rows(float* dst, int L8, const FastDiv& fd_vec, const T* src, int L,
+                                           int nrows, float scale) {
+  const uint32_t nvec = L8 >> 3;
+  const bool vec = (L & 7) == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+  for (uint32_t e = threadIdx.x; e < (uint32_t)nrows * nvec; e += blockDim.x) {
+    const uint32_t r = fd_vec.div(e), c = (e - r * nvec) << 3;
+    float v[8];
+    if (vec) {
+      ldg8(src + (size_t)r * L + c, v);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = (int)c + t < L ? ld_in(src, (size_t)r * L + c + t) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] *= scale;
+    sts8(dst + (size_t)r * L8 + c, v);
+  }
+}
+
+// The 8 fp32 values of one chunk of a lifted row (all zero for a masked residue).
+__device__ __forceinline__ void chunk_values(uint32_t d, bool valid, const float* scal, const float* prow,
+                                             float ptscale, const float* z1row, const float* z2row,
+                                             const float* wrow, int Cz, bool cz8, float (&v)[8]) {
+  const uint32_t src = valid ? (d >> 22) & 15u : (uint32_t)kSrcZero;
+  const int off = d & 2047, woff = (d >> 11) & 2047;
+  if (src == kSrcScalar) {
+    lds8(scal + off, v);
+  } else if (src == kSrcPoint) {
+    lds8(prow + off, v);
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = ptscale * v[t];
+  } else if (src == kSrcPair) {
+    float w[8];
+    lds8(z1row + off, v);
+    if (cz8) {
+      lds8(wrow + woff, w);
+    } else {
+      int cw = woff;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) { w[t] = wrow[cw]; if (++cw == Cz) cw = 0; }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] *= w[t];
+  } else if (src == kSrcZ2) {
+    lds8(z2row + off, v);
+  } else {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = 0.f;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueArgs a) {
   const Plan& p = a.p;
-  const T* q = static_cast<const T*>(a.in.q);
-  const T* k = static_cast<const T*>(a.in.k);
-  const T* v = static_cast<const T*>(a.in.v);
   const T* qp = static_cast<const T*>(a.in.q_pts);
   const T* kp = static_cast<const T*>(a.in.k_pts);
   const T* vp = static_cast<const T*>(a.in.v_pts);
   const T* rot = static_cast<const T*>(a.in.rot);
   const T* tr = static_cast<const T*>(a.in.trans);
-  const T* z1 = static_cast<const T*>(a.in.z1);
-  const T* z2 = static_cast<const T*>(a.in.z2);
   const T* Wb = static_cast<const T*>(a.in.Wb);
   const T* raw = static_cast<const T*>(a.in.raw);
   const int N = p.N, H = p.H, P = p.P, Q = p.Q, Cz = p.Cz, RCz = p.R * p.Cz;
   const int b = blockIdx.y, i0 = blockIdx.x * kLiftRes;
   const int nres = min(kLiftRes, N - i0);
-  const int npt = 2 * P + Q;                 // query, key and value points of one head
+  const int RH = nres * H;
+  const int PW = 2 * p.P38 + p.Q38;            // point row: [a' | b' | g'], each segment zero-padded
+  const int nQ8 = p.Kq >> 3, nK8 = p.KHp >> 3, nV8 = p.VHp >> 3, nZ8 = p.Zp >> 3;
 
-  extern __shared__ float sh[];
-  float* wbt = sh;                                   // [H][Cz]  Wb^T / sqrt(3)
-  float* z1s = wbt + H * Cz;                         // [8][R*Cz]
-  float* z2s = z1s + kLiftRes * RCz;                 // [8][R*Cz]
-  float* pts = z2s + kLiftRes * RCz;                 // [8][H][npt][3]  global point - o_G
-  float* frm = pts + kLiftRes * H * npt * 3;         // [8][12]  R (row-major), t - o_G
-  float* qs = frm + kLiftRes * 12;                   // [8][H][D]
-  float* ks = qs + kLiftRes * H * p.D;               // [8][H][D]
-  float* vs = ks + kLiftRes * H * p.D;               // [8][H][Dv]
+  extern __shared__ float4 sh4[];
+  float* wbt = reinterpret_cast<float*>(sh4);                // [H][Cz]  Wb^T / sqrt(3)
+  float* z1s = wbt + rup(H * Cz, 8);                         // [8][RC8]
+  float* z2s = z1s + kLiftRes * p.RC8;                       // [8][RC8]
+  float* qs = z2s + kLiftRes * p.RC8;                        // [8*H][D8]  q / sqrt(3D)
+  float* ks = qs + kLiftRes * H * p.D8;                      // [8*H][D8]
+  float* vs = ks + kLiftRes * H * p.D8;                      // [8*H][Dv8]
+  float* pts = vs + kLiftRes * H * p.Dv8;                    // [8*H][PW]  global point - o_G
+  float* frm = pts + kLiftRes * H * PW;                      // [8][12]  R (row-major), t - o_G
+  uint32_t* tab = reinterpret_cast<uint32_t*>(frm + kLiftRes * 12);   // chunk descriptors Q | K | V | Z
   __shared__ float s_gamma[64];
   __shared__ int s_valid[kLiftRes];
 
-  // ---- stage every input of the 8 residues (independent loads, issued together)
+  // ---- phase 1: stage the inputs of the 8 residues, zero the point rows,
+  // build the chunk table (independent work, issued together)
   const float inv_sqrt3 = rsqrtf(3.0f);
   const size_t bi0 = (size_t)b * N + i0;
-  for (int e = threadIdx.x; e < H * Cz; e += blockDim.x) {
-    const int h = e / Cz, c = e - h * Cz;
+  for (uint32_t e = threadIdx.x; e < (uint32_t)(H * Cz); e += blockDim.x) {
+    const uint32_t h = p.fd_Cz.div(e), c = e - h * Cz;
     wbt[e] = ld_in(Wb, (size_t)c * H + h) * inv_sqrt3;
   }
-#pragma unroll 4
-  for (int e = threadIdx.x; e < nres * RCz; e += blockDim.x) {
-    z1s[e] = ld_in(z1, bi0 * RCz + e);
-    z2s[e] = ld_in(z2, bi0 * RCz + e);
-  }
-#pragma unroll 4
-  for (int e = threadIdx.x; e < nres * H * p.D; e += blockDim.x) {
-    qs[e] = ld_in(q, bi0 * H * p.D + e);
-    ks[e] = ld_in(k, bi0 * H * p.D + e);
-  }
-#pragma unroll 4
-  for (int e = threadIdx.x; e < nres * H * p.Dv; e += blockDim.x) vs[e] = ld_in(v, bi0 * H * p.Dv + e);
+  stage_rows(z1s, p.RC8, p.fd_RC8v, static_cast<const T*>(a.in.z1) + bi0 * RCz, RCz, nres, 1.f);
+  stage_rows(z2s, p.RC8, p.fd_RC8v, static_cast<const T*>(a.in.z2) + bi0 * RCz, RCz, nres, 1.f);
+  stage_rows(qs, p.D8, p.fd_D8v, static_cast<const T*>(a.in.q) + bi0 * H * p.D, p.D, RH,
+             rsqrtf(3.0f * (float)p.D));
+  stage_rows(ks, p.D8, p.fd_D8v, static_cast<const T*>(a.in.k) + bi0 * H * p.D, p.D, RH, 1.f);
+  stage_rows(vs, p.Dv8, p.fd_Dv8v, static_cast<const T*>(a.in.v) + bi0 * H * p.Dv, p.Dv, RH, 1.f);
+  for (int e = threadIdx.x; e < (RH * PW) >> 2; e += blockDim.x)
+    reinterpret_cast<float4*>(pts)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int e = threadIdx.x; e < nres * 12; e += blockDim.x) {
     const int r = e / 12, c = e - r * 12;
     const size_t bi = bi0 + r;
@@ -134,32 +289,44 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
       frm[e] = ld_in(tr, bi * 3 + (c - 9)) - (c == 9 ? o.x : c == 10 ? o.y : o.z);
     }
   }
+  for (int c = threadIdx.x; c < nQ8 + nK8 + nV8 + nZ8; c += blockDim.x) {
+    int rt = kRowQ, cc = c;
+    if (cc >= nQ8) { cc -= nQ8; rt = kRowK;
+      if (cc >= nK8) { cc -= nK8; rt = kRowV;
+        if (cc >= nV8) { cc -= nV8; rt = kRowZ; } } }
+    tab[c] = chunk_desc(p, rt, cc << 3);
+  }
   for (int h = threadIdx.x; h < H && h < 64; h += blockDim.x) s_gamma[h] = point_weight(ld_in(raw, h), P);
   if (threadIdx.x < nres) s_valid[threadIdx.x] = a.in.mask[bi0 + threadIdx.x] != 0;
   __syncthreads();
 
-  // ---- every point of every head of the 8 residues, relative to its group origin
-#pragma unroll 4
-  for (int e = threadIdx.x; e < nres * H * npt; e += blockDim.x) {
-    const int r = e / (H * npt), rem = e - r * H * npt, h = rem / npt, pt = rem - h * npt;
-    const size_t bih = ((size_t)b * N + i0 + r) * H + h;
-    const T* src = pt < P ? qp + (bih * P + pt) * 3
-                 : pt < 2 * P ? kp + (bih * P + (pt - P)) * 3 : vp + (bih * Q + (pt - 2 * P)) * 3;
-    const float x0 = ld_in(src, 0), x1 = ld_in(src, 1), x2 = ld_in(src, 2);
-    const float* F = frm + r * 12;
-    float* o = pts + (size_t)e * 3;
-    o[0] = F[0] * x0 + F[1] * x1 + F[2] * x2 + F[9];
-    o[1] = F[3] * x0 + F[4] * x1 + F[5] * x2 + F[10];
-    o[2] = F[6] * x0 + F[7] * x1 + F[8] * x2 + F[11];
-  }
+  // ---- phase 2: every point of every head, T_i(x) = R_i x + t_i relative to
+  // the group origin (page "Invariant point attention (IPA)", Required
+  // behavior: column-vector convention)
+  auto apply = [&](const T* src, int npts, const FastDiv& fd_npts, int seg_off) {
+    for (uint32_t e = threadIdx.x; e < (uint32_t)(RH * npts); e += blockDim.x) {
+      const uint32_t rh = fd_npts.div(e), pt = e - rh * npts, r = p.fd_H.div(rh);
+      const T* x = src + ((bi0 * H + rh) * npts + pt) * 3;
+      const float x0 = ld_in(x, 0), x1 = ld_in(x, 1), x2 = ld_in(x, 2);
+      const float* F = frm + r * 12;
+      float* o = pts + (size_t)rh * PW + seg_off + 3 * pt;
+      o[0] = F[0] * x0 + F[1] * x1 + F[2] * x2 + F[9];
+      o[1] = F[3] * x0 + F[4] * x1 + F[5] * x2 + F[10];
+      o[2] = F[6] * x0 + F[7] * x1 + F[8] * x2 + F[11];
+    }
+  };
+  apply(qp, P, p.fd_P, 0);
+  apply(kp, P, p.fd_P, p.P38);
+  apply(vp, Q, p.fd_Q, 2 * p.P38);
   __syncthreads();
 
-  // ---- per (residue, head) fp32 corrections (and the fp32 points of float32 mode)
-  for (int e = threadIdx.x; e < nres * H; e += blockDim.x) {
-    const int r = e / H, h = e - r * H;
+  // ---- phase 3a: per (residue, head) fp32 corrections (and the fp32 points
+  // of float32 mode)
+  for (uint32_t e = threadIdx.x; e < (uint32_t)RH; e += blockDim.x) {
+    const uint32_t r = p.fd_H.div(e), h = e - r * H;
     const float g = s_gamma[h < 64 ? h : 63];
-    const float* pa = pts + (size_t)e * npt * 3;
-    const float* pb = pa + 3 * P;
+    const float* pa = pts + (size_t)e * PW;
+    const float* pb = pa + p.P38;
     float Ax = 0.f, Ay = 0.f, Az = 0.f, a2 = 0.f, Bx = 0.f, By = 0.f, Bz = 0.f, b2 = 0.f;
     for (int pp = 0; pp < P; ++pp) {
       Ax += pa[3 * pp]; Ay += pa[3 * pp + 1]; Az += pa[3 * pp + 2];
@@ -182,122 +349,41 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     }
   }
 
-  // ---- every lifted row as 16-byte chunks (8 fp16 values of one segment):
-  // one warp per row, lanes over its chunks
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarp = blockDim.x >> 5;
-  const float sqk = rsqrtf(3.0f * (float)p.D);
-  const int sq = p.nsq * p.D8;          // scalar columns of the query / key head part
-  const int sv = p.nsv * p.Dv8;         // scalar columns of the value head part
-  for (int row = warp; row < nres * H; row += nwarp) {
-    const int r = row / H, h = row - r * H, i = i0 + r;
-    const bool valid = s_valid[r] != 0;
-    const float* qsr = qs + (r * H + h) * p.D;
-    const float* ksr = ks + (r * H + h) * p.D;
-    const float* vsr = vs + (r * H + h) * p.Dv;
-    const float* pa = pts + ((size_t)r * H + h) * npt * 3;
-    const float* pb = pa + 3 * P;
-    const float* pg = pb + 3 * P;
-    const float g2 = 2.f * s_gamma[h < 64 ? h : 63];
-    const size_t rowid = ((size_t)b * H + h) * N + i;
-    // query row: [ scalar | points (tensor-core mode) | pad ] [ pair part ]
-    __half* qrow = a.w.Q + rowid * p.Kq;
-    for (int c8 = lane; c8 < p.Kq / 8; c8 += 32) {
-      const int col = c8 * 8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      bool lo = false;
-      if (valid) {
-        if (col < sq) {
-          const int seg = col / p.D8, e0 = col - seg * p.D8;
-          lo = (seg == 2);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) if (e0 + t < p.D) v[t] = qsr[e0 + t] * sqk;
-        } else if (col < p.KHp) {
-          if (!p.geo_simt && col < sq + 3 * p.P38) {
-            const int seg = (col - sq) / p.P38, e0 = col - sq - seg * p.P38;
-            lo = (seg == 2);
-#pragma unroll
-            for (int t = 0; t < 8; ++t) if (e0 + t < 3 * P) v[t] = g2 * pa[e0 + t];
-          }
-        } else {
-          const int cc = col - p.KHp;
-          int e0;
-          if (p.nqz == 2) {                        // [u hi | u lo], each Zp wide
-            lo = cc >= p.Zp;
-            e0 = lo ? cc - p.Zp : cc;
-          } else {                                 // [u hi | u hi | u lo], RC8 apart
-            const int seg = cc / p.RC8;
-            e0 = seg < p.nz ? cc - seg * p.RC8 : RCz;
-            lo = (seg == 2);
-          }
-          if (e0 < RCz) {
-            int rr = e0 / Cz, c0 = e0 - rr * Cz;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              if (e0 + t < RCz) v[t] = z1s[r * RCz + e0 + t] * wbt[h * Cz + c0];
-              if (++c0 == Cz) { c0 = 0; ++rr; }
-            }
-          }
-        }
-      }
-      store8(qrow + col, v, lo);
-    }
-    // key row (head part): [ scalar | points (tensor-core mode) | pad ]
-    __half* krow = a.w.KH + rowid * p.KHp;
-    for (int c8 = lane; c8 < p.KHp / 8; c8 += 32) {
-      const int col = c8 * 8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      bool lo = false;
-      if (valid) {
-        if (col < sq) {
-          const int seg = col / p.D8, e0 = col - seg * p.D8;
-          lo = (seg == 1);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) if (e0 + t < p.D) v[t] = ksr[e0 + t];
-        } else if (!p.geo_simt && col < sq + 3 * p.P38) {
-          const int seg = (col - sq) / p.P38, e0 = col - sq - seg * p.P38;
-          lo = (seg == 1);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) if (e0 + t < 3 * P) v[t] = pb[e0 + t];
-        }
-      }
-      store8(krow + col, v, lo);
-    }
-    // value row (head part): [ scalar | g' hi | g' lo | pad ]
-    __half* vrow = a.w.VH + rowid * p.VHp;
-    for (int c8 = lane; c8 < p.VHp / 8; c8 += 32) {
-      const int col = c8 * 8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      bool lo = false;
-      if (valid) {
-        if (col < sv) {
-          const int seg = col / p.Dv8, e0 = col - seg * p.Dv8;
-          lo = (seg == 1);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) if (e0 + t < p.Dv) v[t] = vsr[e0 + t];
-        } else if (col < sv + 2 * p.Q38) {
-          const int seg = (col - sv) / p.Q38, e0 = col - sv - seg * p.Q38;
-          lo = (seg == 1);
-#pragma unroll
-          for (int t = 0; t < 8; ++t) if (e0 + t < 3 * Q) v[t] = pg[e0 + t];
-        }
-      }
-      store8(vrow + col, v, lo);
-    }
+  // ---- phase 3b: every lifted row, one pass per row type over all (row,
+  // chunk) pairs of the CTA: consecutive threads write consecutive 16-byte
+  // chunks of a row
+  const bool cz8 = (Cz & 7) == 0;
+  const uint32_t nthr = blockDim.x;
+  for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nQ8; e += nthr) {
+    const uint32_t rh = p.fd_nQ8.div(e), c = e - rh * nQ8, r = p.fd_H.div(rh), h = rh - r * H;
+    const uint32_t d = tab[c];
+    float v[8];
+    chunk_values(d, s_valid[r] != 0, qs + (size_t)rh * p.D8, pts + (size_t)rh * PW, 2.f * s_gamma[h < 64 ? h : 63],
+                 z1s + (size_t)r * p.RC8, nullptr, wbt + (size_t)h * Cz, Cz, cz8, v);
+    stg8_half(a.w.Q + (((size_t)b * H + h) * N + i0 + r) * p.Kq + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
-  // pair factor rows z2 (shared by the heads): [ z2 segments | pad ]
-  for (int r = warp; r < nres; r += nwarp) {
-    const bool valid = s_valid[r] != 0;
-    __half* zrow = a.w.Z + (bi0 + r) * p.Zp;
-    for (int c8 = lane; c8 < p.Zp / 8; c8 += 32) {
-      const int col = c8 * 8, seg = col / p.RC8, e0 = col - seg * p.RC8;
-      float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const bool lo = (seg == 1);
-      if (valid && seg < p.nz) {
-#pragma unroll
-        for (int t = 0; t < 8; ++t) if (e0 + t < RCz) v[t] = z2s[r * RCz + e0 + t];
-      }
-      store8(zrow + col, v, lo);
-    }
+  for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nK8; e += nthr) {
+    const uint32_t rh = p.fd_nK8.div(e), c = e - rh * nK8, r = p.fd_H.div(rh), h = rh - r * H;
+    const uint32_t d = tab[nQ8 + c];
+    float v[8];
+    chunk_values(d, s_valid[r] != 0, ks + (size_t)rh * p.D8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr,
+                 nullptr, Cz, cz8, v);
+    stg8_half(a.w.KH + (((size_t)b * H + h) * N + i0 + r) * p.KHp + ((size_t)c << 3), v, (d >> 26) & 1u);
+  }
+  for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nV8; e += nthr) {
+    const uint32_t rh = p.fd_nV8.div(e), c = e - rh * nV8, r = p.fd_H.div(rh), h = rh - r * H;
+    const uint32_t d = tab[nQ8 + nK8 + c];
+    float v[8];
+    chunk_values(d, s_valid[r] != 0, vs + (size_t)rh * p.Dv8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr,
+                 nullptr, Cz, cz8, v);
+    stg8_half(a.w.VH + (((size_t)b * H + h) * N + i0 + r) * p.VHp + ((size_t)c << 3), v, (d >> 26) & 1u);
+  }
+  for (uint32_t e = threadIdx.x; e < (uint32_t)nres * nZ8; e += nthr) {
+    const uint32_t r = p.fd_nZ8.div(e), c = e - r * nZ8;
+    const uint32_t d = tab[nQ8 + nK8 + nV8 + c];
+    float v[8];
+    chunk_values(d, s_valid[r] != 0, nullptr, nullptr, 1.f, nullptr, z2s + (size_t)r * p.RC8, nullptr, Cz, cz8, v);
+    stg8_half(a.w.Z + (bi0 + r) * p.Zp + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
 }
 
