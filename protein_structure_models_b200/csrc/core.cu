@@ -167,7 +167,7 @@ __device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col,
 // shared memory); (Gx,Gy,Gz) = sum_j a_ij o_G(j), the group-origin part of
 // the aggregated value points.  Also writes local_points.
 __device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, float* orow, float Gx, float Gy,
-                               float Gz, bool with_pair) {
+                               float Gz, bool with_pair, const float (&R)[9], const float (&t)[3]) {
   const Plan& p = a.p;
   const int H = p.H, Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.F;
   __half* frow = a.feat + bi * p.Kgp;
@@ -183,11 +183,6 @@ __device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, 
     for (int e = 0; e < 3 * Q; ++e) lp[e] = 0.f;
     return;
   }
-  float R[9], t[3];
-#pragma unroll
-  for (int e = 0; e < 9; ++e) R[e] = ld_any(a.rot, bi * 9 + e, p.f32);
-#pragma unroll
-  for (int e = 0; e < 3; ++e) t[e] = ld_any(a.trans, bi * 3 + e, p.f32);
   // scalar block
   put_run(frow, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
   // points: aggregate (hi + lo halves + group-origin part), back into the query
@@ -239,6 +234,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Plan& p = a.p;
+  // CTA timeline (debug trace only): the last 8 slots of the softmax role's log
+  const bool timeline = a.trace != nullptr && threadIdx.x == 128 &&
+                        (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) == a.trace_cta;
+  Tracer ttr{timeline ? a.trace + (size_t)2 * 2 * kTraceCap : nullptr, kTraceCap - 8};
+  ttr.ev(40);
   uint8_t* sQ = smem;
   uint8_t* sRing = sQ + p.nQc * kChunkBytes;
   uint8_t* tail = sRing + p.nst * kChunkBytes;
@@ -300,12 +300,22 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const int nkt = *ntiles;
   const WaitCtx wc{abort_flag, a.status, a.timeout_ns};
+  ttr.ev(41);
   const int lin_cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
   long long* tbase = (a.trace != nullptr && lin_cta == a.trace_cta) ? a.trace : nullptr;
   auto tracer = [&](int role) { return Tracer{tbase ? tbase + (size_t)role * 2 * kTraceCap : nullptr, 0}; };
   // per-row softmax state, read by the fused feature epilogue after the roles end
   float rowM = -INFINITY, rowL = 0.f, rowW[3] = {0.f, 0.f, 0.f};
   bool row_ok = false;
+  float rowR[9], rowT[3];   // frame of the row's residue, loaded during the last tile
+  // z1 rows of the query tile, prefetched into the dead Qhat buffer once the
+  // last logit tile has been read (row stride padded by 16 bytes)
+  const size_t z1_row_bytes = (size_t)p.R * p.Cz * (p.f32 ? 4 : 2);
+  const size_t z1_stride = z1_row_bytes + 16;
+  const size_t z1_off = ((size_t)kTile * (p.VHp + 1) * 4 + 1023) & ~(size_t)1023;
+  const bool fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(a.z1) & 15) == 0;
+  const bool z1_smem = fast_pair && (z1_row_bytes & 15) == 0 &&
+                       z1_off + kTile * z1_stride <= (size_t)p.nQc * kChunkBytes;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -364,7 +374,6 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       int st = 0;
       uint32_t ph = 0;
       const uint32_t idS = idesc_f16(128, 128, 0, 0);
-      const uint32_t idO = idesc_f16(128, 64, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
       auto mma_qk = [&]() -> bool {
         // key chunks in ring order: the pair part first (each z2 chunk meets nqz
@@ -395,22 +404,32 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         return true;
       };
       auto mma_pv = [&](int s) -> bool {
+        // value chunks in O-column order; up to 4 chunks in consecutive ring
+        // slots form one MMA of N = 64 x run (MN-major B, groups 16 KB apart)
         const int nchunk = p.nVH + p.nZV;
-        for (int c = 0; c < nchunk; ++c) {
-          tr.ev(11);
-          if (!mbar_wait(&full[st], ph, wc, 4)) return false;
-          tr.ev(12);
+        for (int c = 0; c < nchunk;) {
+          int run = nchunk - c;
+          if (run > 4) run = 4;
+          if (run > p.nst - st) run = p.nst - st;
+          for (int u = 0; u < run; ++u) {
+            tr.ev(11);
+            if (!mbar_wait(&full[st + u], ph, wc, 4)) return false;
+            tr.ev(12);
+          }
           tc_fence_after();
           const uint32_t b0 = sRa + st * kChunkBytes;
           const uint32_t dcol = tmem + (uint32_t)(p.tmemO + c * kChunk);
+          const uint32_t idO = idesc_f16(128, 64 * run, 0, 1);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t bd = desc_mnmajor_sw128(b0 + kk * 2048, kChunkBytes);
             mma_ts(dcol, tmem + kTmemP + kk * 8, bd, idO, (s > 0 || kk > 0) ? 1u : 0u);
             if (SPLIT) mma_ts(dcol, tmem + kTmemP + 64 + kk * 8, bd, idO, 1u);
           }
-          tc_commit(&empty[st]);
-          if (++st == p.nst) { st = 0; ph ^= 1u; }
+          for (int u = 0; u < run; ++u) tc_commit(&empty[st + u]);
+          st += run;
+          if (st == p.nst) { st = 0; ph ^= 1u; }
+          c += run;
         }
         tc_commit(pv_done);
         tr.ev(18);
@@ -657,6 +676,23 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       mbar_arrive(p_full);
       str.ev(26);
     }
+    {
+      // every QK^T product has completed (the last logits were read), so the
+      // Qhat buffer is free: prefetch this row's z1 factors and frame while the
+      // last P.V product runs
+      const int i = qt * kTile + wq * 32 + lane;
+      const size_t bi = (size_t)b * N + (i < N ? i : 0);
+#pragma unroll
+      for (int e = 0; e < 9; ++e) rowR[e] = ld_any(a.rot, bi * 9 + e, p.f32);
+#pragma unroll
+      for (int e = 0; e < 3; ++e) rowT[e] = ld_any(a.trans, bi * 3 + e, p.f32);
+      if (z1_smem && i < N) {
+        const uint8_t* src = static_cast<const uint8_t*>(a.z1) + bi * z1_row_bytes;
+        uint8_t* dst = smem + z1_off + (size_t)(wq * 32 + lane) * z1_stride;
+        for (size_t o = 0; o < z1_row_bytes; o += 16) cp_async16(dst + o, src + o);
+      }
+      cp_async_commit();
+    }
     if (ok && nkt > 0) {
       ok = mbar_wait(pv_done, (nkt - 1) & 1, wc, 9);
       ok = __all_sync(0xffffffffu, ok);
@@ -676,13 +712,13 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  ttr.ev(42);
   if (warp >= 4 && *abort_flag == 0) {
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const int i = qt * kTile + r;
     const bool in_range = i < N;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
-    const bool fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(a.z1) & 15) == 0;
     const int staged = fast_pair ? p.VHp : p.Ocols;         // columns staged in shared memory
     float* orow = reinterpret_cast<float*>(smem) + (size_t)r * (staged + 1);
     const float inv = rowL > 0.f ? 1.f / rowL : 0.f;
@@ -696,6 +732,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv;
       }
     }
+    ttr.ev(45);
     const size_t bi = (size_t)b * N + (in_range ? i : 0);
     const bool empty = !(rowL > 0.f) || !live;
     if (in_range) {
@@ -705,12 +742,15 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         a.lse[(size_t)bh * N + i] = rowL > 0.f ? (rowM + log2f(rowL)) * kLn2 + qv.w : -INFINITY;
       }
       if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
-      write_features(a, bi, h, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair);
+      write_features(a, bi, h, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT);
     }
+    ttr.ev(46);
     if (fast_pair) {
       // pair block straight from tensor memory, 32 channels at a time
       const int Cz = p.Cz, RCz = p.R * Cz, pcol = p.H * p.Dv + 4 * p.H * p.Q + h * Cz;
       __half* frow = a.feat + bi * p.Kgp;
+      cp_async_wait_all();
+      const uint8_t* zs = smem + z1_off + (size_t)r * z1_stride;
       for (int c0 = 0; c0 < Cz; c0 += 32) {
         float acc[32];
 #pragma unroll
@@ -730,19 +770,22 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           }
           if (in_range && !empty) {
             const size_t zoff = bi * RCz + (size_t)rr * Cz + c0;
+            const size_t zrel = (size_t)rr * Cz + c0;
             float zv[32];
             if (p.f32) {
-              const float4* z4 = reinterpret_cast<const float4*>(static_cast<const float*>(a.z1) + zoff);
+              const float4* z4 = z1_smem ? reinterpret_cast<const float4*>(zs) + zrel / 4
+                                         : reinterpret_cast<const float4*>(static_cast<const float*>(a.z1) + zoff);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
-                const float4 t4 = __ldg(z4 + k);
+                const float4 t4 = z1_smem ? z4[k] : __ldg(z4 + k);
                 zv[4 * k] = t4.x; zv[4 * k + 1] = t4.y; zv[4 * k + 2] = t4.z; zv[4 * k + 3] = t4.w;
               }
             } else {
-              const uint4* z4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z1) + zoff);
+              const uint4* z4 = z1_smem ? reinterpret_cast<const uint4*>(zs) + zrel / 8
+                                        : reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z1) + zoff);
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const uint4 t4 = __ldg(z4 + k);
+                const uint4 t4 = z1_smem ? z4[k] : __ldg(z4 + k);
                 const uint32_t w4[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -758,11 +801,14 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (in_range) put_run32(frow, p.F, p.f32, pcol + c0, acc);
       }
     }
+    ttr.ev(47);
   }
 
   // ---------------------------------------------------------------- teardown
+  ttr.ev(43);
   tc_fence_before();
   __syncthreads();
+  ttr.ev(44);
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
