@@ -141,26 +141,69 @@ def measured_peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
-def core_source_hash() -> str:
+# Sources of each timed kernel; a committed ncu summary counts only while its
+# recorded hash of these files matches.
+KERNEL_SOURCES = {
+    "fipa_lift_kernel": ("prologue.cu", "sm100.cuh", "plan.h", "kernels.h"),
+    "fipa_core_kernel": ("core.cu", "sm100.cuh", "plan.h", "kernels.h"),
+    "fipa_out_proj_kernel": ("epilogue.cu", "sm100.cuh", "plan.h", "kernels.h"),
+}
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in ("core.cu", "sm100.cuh", "plan.h"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "protein_structure_models_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(wl):
-    """DRAM bytes per core launch from a committed ncu summary, if it was taken
-    on the current core kernel source for this workload."""
-    path = os.path.join(ROOT, "profiles", f"fipa_core_kernel-{wl.name}.md")
+def profiled_traffic(kernel: str, wl):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, if it
+    was taken on the current source of that kernel for this workload."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}-{wl.name}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m_h = re.search(r"core_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
     m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", text)
-    if not m_h or not m_b or m_h.group(1) != core_source_hash():
+    if not m_h or not m_b or m_h.group(1) != source_hash(kernel):
         return None
     return int(m_b.group(1))
+
+
+def _rup(a, b):
+    return (a + b - 1) // b * b
+
+
+def lifted_widths(wl):
+    """Column widths of the lifted fp16 rows the prologue writes (the layout of
+    csrc/plan.h): Qhat Kq, key head part KHp, value head part VHp, pair rows Zp."""
+    f32 = wl.dtype == "f32"
+    nsq, nsv, nz, nqz = (3, 2, 3, 1) if f32 else (1, 1, 1, 2)
+    D8, P38, Dv8, Q38, RC8 = _rup(wl.D, 8), _rup(3 * wl.P, 8), _rup(wl.Dv, 8), _rup(3 * wl.Q, 8), _rup(wl.R * wl.Cz, 8)
+    KHp = _rup(nsq * D8 + (0 if f32 else 3 * P38), 64)
+    Zp = _rup(nz * RC8, 64)
+    return {"Kq": KHp + nqz * Zp, "KHp": KHp, "VHp": _rup(nsv * Dv8 + 2 * Q38, 64), "Zp": Zp}
+
+
+def prologue_bytes(wl) -> int:
+    """Bytes the prologue must move: every input it reads once, and the lifted
+    rows plus per-row fp32 vectors it writes."""
+    es = 4 if wl.dtype == "f32" else 2
+    BN, BHN = wl.B * wl.N, wl.B * wl.H * wl.N
+    reads = es * (BHN * (2 * wl.D + wl.Dv + 6 * wl.P + 3 * wl.Q) + BN * (12 + 2 * wl.R * wl.Cz)) + BN
+    w = lifted_widths(wl)
+    writes = 2 * (BHN * (w["Kq"] + w["KHp"] + w["VHp"]) + BN * w["Zp"]) + 32 * BHN
+    if wl.dtype == "f32":
+        writes += 2 * BHN * 3 * wl.P * 4
+    return int(reads + writes)
+
+
+def out_proj_flops(wl) -> int:
+    """Algorithmic flops of update = features @ w_out over all B*N rows."""
+    F = wl.H * (wl.Dv + 4 * wl.Q + wl.Cz)
+    return 2 * wl.B * wl.N * F * wl.Cout
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
@@ -297,6 +340,35 @@ def run_fipa(args, wl, rank, world, local_rank):
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
 
 
+def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src):
+    """Achieved rate of each timed kernel against its roofline; the time of a
+    kernel is its stage's mean CUDA-event time inside the timed steps."""
+    lift_s = stage_ms["prologue"] / 1e3
+    core_s = stage_ms["core"] / 1e3
+    proj_s = stage_ms["out_proj"] / 1e3
+    pb, pf, cf = prologue_bytes(wl), out_proj_flops(wl), valid * fpp
+    tensor_peak = f"{src} bf16 dense burst, {burst} TFLOP/s (fp16 operands run at the bf16 rate)"
+    return {
+        "fipa_lift_kernel": {
+            "bound": "hbm", "achieved": pb / lift_s / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": pb / lift_s / 1e9 / hbm, "peak_source": f"{src} HBM copy bandwidth",
+            "work": f"{pb} bytes per launch (inputs read once + lifted rows written); "
+                    f"time = prologue stage (origin + lift kernels)",
+            "traffic": profiled_traffic("fipa_lift_kernel", wl)},
+        "fipa_core_kernel": {
+            "bound": "tensor", "achieved": cf / core_s / 1e12, "peak": burst, "unit": "TFLOP/s",
+            "frac": cf / core_s / 1e12 / burst, "peak_source": tensor_peak,
+            "frac_of_datasheet_2250": cf / core_s / 1e12 / 2250.0,
+            "work": f"{fpp} flop per valid (b,h,i,j) x {valid} valid pairs per launch",
+            "traffic": profiled_traffic("fipa_core_kernel", wl)},
+        "fipa_out_proj_kernel": {
+            "bound": "tensor", "achieved": pf / proj_s / 1e12, "peak": burst, "unit": "TFLOP/s",
+            "frac": pf / proj_s / 1e12 / burst, "peak_source": tensor_peak,
+            "work": f"2*F*Cout flop x B*N rows = {pf} per launch; time = out_proj stage",
+            "traffic": profiled_traffic("fipa_out_proj_kernel", wl)},
+    }
+
+
 def main_fipa(args, wl):
     rank, world, local_rank = dist_info()
     if world > 1:
@@ -312,9 +384,11 @@ def main_fipa(args, wl):
     padded, valid = pair_counts(wl, inp)
     fpp = flops_per_pair(wl)
     burst, sustained, hbm, src = measured_peaks()
-    core_s = r["core_ms"] / 1e3
-    achieved = valid * fpp / core_s / 1e12
     value = padded * world / (r["step_ms"] / 1e3)
+    kernels = kernel_rooflines(wl, r["stage_ms"], valid, fpp, burst, hbm, src)
+    stage_of = {"fipa_lift_kernel": "prologue", "fipa_core_kernel": "core", "fipa_out_proj_kernel": "out_proj"}
+    dominant = max(kernels, key=lambda k: r["stage_ms"][stage_of[k]])
+    roofline = dict(kernels[dominant], kernel=dominant)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         rate, done, el = cpu_oracle_rate(wl, inp, args.cpu_seconds)
@@ -329,11 +403,8 @@ def main_fipa(args, wl):
                                        "math": "fp16 tensor-core products, fp32 accumulate; bf16 inputs"}),
         "valid_pairs_per_s": valid * world / (r["step_ms"] / 1e3),
         "stage_ms": r["stage_ms"],
-        "roofline": {"kernel": "fipa_core_kernel", "bound": "tensor", "achieved": achieved,
-                     "peak": burst, "unit": "TFLOP/s", "frac": achieved / burst,
-                     "peak_source": f"{src} bf16 dense burst (fp16 nominal rate = bf16)",
-                     "work": f"{fpp} flop per valid (b,h,i,j) x {valid} valid pairs per launch",
-                     "traffic": profiled_traffic(wl)},
+        "roofline": roofline,
+        "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": {"value": padded * world / (r["e2e_ms"] / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
