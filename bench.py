@@ -232,6 +232,11 @@ def blas_threads():
 
 
 # ---------------------------------------------------------------- GPU arm
+def replica_seed(wl, rank: int) -> int:
+    """Seed of rank `rank`'s replica: rank 0 runs the workload's own inputs."""
+    return wl.seed + 1000 * rank
+
+
 def to_device(inp, dtype, dev):
     import torch
     td = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -249,10 +254,11 @@ def run_fipa(args, wl, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     from protein_structure_models_b200 import Fipa
+    from protein_structure_models_b200.sharding import max_over_ranks
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    inp = workloads.make_inputs(wl, seed=wl.seed + 1000 * rank)
+    inp = workloads.make_inputs(wl, seed=replica_seed(wl, rank))
     d_in = to_device(inp, wl.dtype, dev)
     h = Fipa(wl.dtype, local_rank)
     dims = wl.dims()
@@ -305,10 +311,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     del graph
     step_ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
     core_ms = stage_sum["core"] / args.steps
-    t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t.item())
+    step_ms_max = max_over_ranks(step_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs -> device -> result on host
     host_in = {k: v.cpu().pin_memory() for k, v in d_in.items() if v is not None}
@@ -329,10 +332,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h.sync_status()
     h.close()
     return dict(inp=inp, step_ms=step_ms_max, core_ms=core_ms, launches=launches,
