@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="length sweep N=512..16384: time, peak memory, fitted exponents (JSON lines)")
     return ap.parse_args()
 
 
@@ -462,8 +464,95 @@ def main_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def fit_loglog(ns, ts):
+    """Least-squares exponent of log t against log N with its 95% confidence
+    interval (Student t, n - 2 degrees of freedom)."""
+    from scipy import stats
+    x, y = np.log(np.asarray(ns, float)), np.log(np.asarray(ts, float))
+    n = len(x)
+    A = np.vstack([x, np.ones(n)]).T
+    (slope, icpt), *_ = np.linalg.lstsq(A, y, rcond=None)
+    resid = y - (slope * x + icpt)
+    dof = n - 2
+    se = float(np.sqrt(resid @ resid / dof / np.sum((x - x.mean()) ** 2))) if dof > 0 else float("nan")
+    half = float(stats.t.ppf(0.975, dof)) * se if dof > 0 else float("nan")
+    return {"exponent": float(slope), "ci95": [float(slope - half), float(slope + half)], "points": n}
+
+
+def fit_linear(ns, ys):
+    """Least-squares line y = a N + c and its R^2."""
+    x, y = np.asarray(ns, float), np.asarray(ys, float)
+    a, c = np.polyfit(x, y, 1)
+    pred = a * x + c
+    ss = float(np.sum((y - y.mean()) ** 2))
+    r2 = 1.0 - float(np.sum((y - pred) ** 2)) / ss if ss > 0 else 1.0
+    return {"bytes_per_residue": float(a), "intercept_bytes": float(c), "r2": r2}
+
+
+def main_sweep(args):
+    """Length sweep: per N the graph-timed forward, and the peak device bytes
+    held by inputs, outputs and workspace (torch's peak counter, reset before
+    they are allocated); then the exponent of time vs N and the line of
+    memory vs N.  One JSON line per N, then one with the fits."""
+    import torch
+    from protein_structure_models_b200 import Fipa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ns, ts, mems = [], [], []
+    for N in workloads.SWEEP_N:
+        wl = workloads.workload(f"3-{N}")
+        inp = workloads.make_inputs(wl)
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        d_in = to_device(inp, wl.dtype, dev)
+        h = Fipa(wl.dtype, 0)
+        ws = torch.empty(h.workspace_size(wl.dims()), dtype=torch.uint8, device=dev)
+        out = {"update": torch.empty((wl.B, wl.N, wl.Cout), dtype=torch.float32, device=dev),
+               "local_points": torch.empty((wl.B, wl.N, wl.H, wl.Q, 3), dtype=torch.float32, device=dev)}
+        stream = torch.cuda.current_stream(dev)
+        h.forward(d_in, eps=inp["eps"], workspace=ws, out=out, stream=stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            h.forward(d_in, eps=inp["eps"], workspace=ws, out=out, stream=cap)
+        torch.cuda.synchronize()
+        steps = max(5, min(200, int(2000 * 512 * 512 / N ** 2)))
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            graph.replay()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for k in range(steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            graph.replay()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        h.sync_status()
+        ms = float(np.median([a.elapsed_time(b) for a, b in ev]))
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        del graph
+        h.close()
+        ns.append(N); ts.append(ms); mems.append(peak)
+        print(json.dumps({"sweep": "length", "N": N, "ms_per_forward": ms, "steps": steps,
+                          "pairs_per_s": wl.B * wl.H * N * N / (ms / 1e3), "peak_device_bytes": int(peak),
+                          "workspace_bytes": int(ws.numel())}), flush=True)
+        del d_in, ws, out
+        torch.cuda.empty_cache()
+    big = [i for i, n in enumerate(ns) if n >= 2048]
+    print(json.dumps({"sweep": "length", "fit_time_all": fit_loglog(ns, ts),
+                      "fit_time_N_ge_2048": fit_loglog([ns[i] for i in big], [ts[i] for i in big]),
+                      "fit_memory": fit_linear(ns, mems)}), flush=True)
+
+
 def main():
     args = parse_args()
+    if args.sweep:
+        main_sweep(args)
+        return
     wl = workloads.workload(args.workload)
     if args.impl == "reference":
         main_reference(args, wl)

@@ -1,0 +1,43 @@
+"""Host-side fits of the length sweep in bench.py."""
+import os
+import sys
+
+import numpy as np
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+import bench  # noqa: E402
+
+
+def test_loglog_exact_power_law():
+    ns = [512, 1024, 2048, 4096, 8192, 16384]
+    ts = [3e-7 * n ** 1.7 for n in ns]
+    f = bench.fit_loglog(ns, ts)
+    assert abs(f["exponent"] - 1.7) < 1e-12
+    assert abs(f["ci95"][0] - 1.7) < 1e-9 and abs(f["ci95"][1] - 1.7) < 1e-9
+
+
+def test_loglog_interval_contains_slope_with_noise():
+    rng = np.random.default_rng(1)
+    ns = np.array([512, 1024, 2048, 4096, 8192, 16384])
+    ts = 1e-6 * ns ** 2.0 * np.exp(rng.normal(0, 0.05, ns.size))
+    f = bench.fit_loglog(ns, ts)
+    assert f["ci95"][0] < f["exponent"] < f["ci95"][1]
+    assert f["ci95"][0] < 2.0 < f["ci95"][1]
+
+
+def test_linear_memory_fit():
+    ns = [512, 1024, 4096]
+    f = bench.fit_linear(ns, [1000 + 20 * n for n in ns])
+    assert abs(f["bytes_per_residue"] - 20) < 1e-9 and abs(f["intercept_bytes"] - 1000) < 1e-6
+    assert abs(f["r2"] - 1.0) < 1e-12
+
+
+def test_prologue_bytes_matches_hand_count_for_protein_batch():
+    import workloads
+    wl = workloads.workload("1")
+    w = bench.lifted_widths(wl)
+    assert w == {"Kq": 576, "KHp": 64, "VHp": 64, "Zp": 256}
+    BN, BHN = 8 * 256, 8 * 8 * 256
+    reads = 2 * (BHN * (32 + 16 + 24 + 24) + BN * (12 + 512)) + BN
+    writes = 2 * (BHN * (576 + 64 + 64) + BN * 256) + 32 * BHN
+    assert bench.prologue_bytes(wl) == reads + writes
