@@ -84,79 +84,61 @@ __device__ __forceinline__ float ld_any(const void* ptr, size_t i, int f32) {
              : __bfloat162float(static_cast<const __nv_bfloat16*>(ptr)[i]);
 }
 
-__device__ __forceinline__ uint32_t half2_bits(__half a, __half b) {
-  return (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
-}
 
-// Feature values val(0..n-1) at feature columns [col, col+n) of the projection
-// operand row: fp16 hi at col and lo at F+col (float32 inputs: hi, hi, lo at
-// col, F+col, 2F+col).  16-byte stores where the run is aligned.
-template <typename Fn>
-__device__ __forceinline__ void put_run(__half* frow, int F, int f32, int col, int n, Fn&& val) {
-  for (int k0 = 0; k0 < n; k0 += 8) {
-    float v[8];
+// 8 feature values at columns [c, c+8) of one head block of the projection
+// operand: fp16 hi at c and the residual lo = fp16(x - hi) at F+c, F the
+// segment stride (float32 inputs: hi, hi, lo at c, F+c, 2F+c); n <= 8 of them
+// are stored.  One 16-byte store per segment where the run is aligned.
+__device__ __forceinline__ void put8(__half* frow, int F, int f32, int c, int n, const float (&v)[8]) {
+  uint32_t hw[4], lw[4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) v[t] = k0 + t < n ? val(k0 + t) : 0.f;
-    __half hi[8], lo[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      hi[t] = __float2half_rn(v[t]);
-      lo[t] = __float2half_rn(v[t] - __half2float(hi[t]));
-    }
-    const int c = col + k0;
-    if (k0 + 8 <= n && (c & 7) == 0 && (F & 7) == 0) {
-      const uint4 H4 = make_uint4(half2_bits(hi[0], hi[1]), half2_bits(hi[2], hi[3]), half2_bits(hi[4], hi[5]),
-                                  half2_bits(hi[6], hi[7]));
-      const uint4 L4 = make_uint4(half2_bits(lo[0], lo[1]), half2_bits(lo[2], lo[3]), half2_bits(lo[4], lo[5]),
-                                  half2_bits(lo[6], lo[7]));
-      *reinterpret_cast<uint4*>(frow + c) = H4;
-      if (f32) {
-        *reinterpret_cast<uint4*>(frow + F + c) = H4;
-        *reinterpret_cast<uint4*>(frow + 2 * F + c) = L4;
-      } else {
-        *reinterpret_cast<uint4*>(frow + F + c) = L4;
-      }
+  for (int t = 0; t < 4; ++t) {
+    const __half2 h = __floats2half2_rn(v[2 * t], v[2 * t + 1]);
+    const float2 f = __half22float2(h);
+    const __half2 l = __floats2half2_rn(v[2 * t] - f.x, v[2 * t + 1] - f.y);
+    hw[t] = *reinterpret_cast<const uint32_t*>(&h);
+    lw[t] = *reinterpret_cast<const uint32_t*>(&l);
+  }
+  if (n == 8 && ((c | F) & 7) == 0) {
+    const uint4 H4 = make_uint4(hw[0], hw[1], hw[2], hw[3]), L4 = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    *reinterpret_cast<uint4*>(frow + c) = H4;
+    if (f32) {
+      *reinterpret_cast<uint4*>(frow + F + c) = H4;
+      *reinterpret_cast<uint4*>(frow + 2 * F + c) = L4;
     } else {
-      for (int t = 0; t < 8 && k0 + t < n; ++t) {
-        frow[c + t] = hi[t];
-        if (f32) { frow[F + c + t] = hi[t]; frow[2 * F + c + t] = lo[t]; }
-        else     { frow[F + c + t] = lo[t]; }
-      }
+      *reinterpret_cast<uint4*>(frow + F + c) = L4;
+    }
+  } else {
+    const __half* hh = reinterpret_cast<const __half*>(hw);
+    const __half* ll = reinterpret_cast<const __half*>(lw);
+    for (int t = 0; t < n; ++t) {
+      frow[c + t] = hh[t];
+      if (f32) { frow[F + c + t] = hh[t]; frow[2 * F + c + t] = ll[t]; }
+      else     { frow[F + c + t] = ll[t]; }
     }
   }
 }
 
-// 32 feature values from registers at columns [col, col+32), as put_run.
+// Feature values val(0..n-1) at columns [col, col+n), as put8.
+template <typename Fn>
+__device__ __forceinline__ void put_run(__half* frow, int F, int f32, int col, int n, Fn&& val) {
+  for (int k0 = 0; k0 < n; k0 += 8) {
+    const int m = min(8, n - k0);
+    float v[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = t < m ? val(k0 + t) : 0.f;
+    put8(frow, F, f32, col + k0, m, v);
+  }
+}
+
+// 32 feature values from registers at columns [col, col+32), as put8.
 __device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col, const float (&v)[32]) {
 #pragma unroll
   for (int k0 = 0; k0 < 32; k0 += 8) {
-    __half hi[8], lo[8];
+    float w[8];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      hi[t] = __float2half_rn(v[k0 + t]);
-      lo[t] = __float2half_rn(v[k0 + t] - __half2float(hi[t]));
-    }
-    const int c = col + k0;
-    if ((c & 7) == 0 && (F & 7) == 0) {
-      const uint4 H4 = make_uint4(half2_bits(hi[0], hi[1]), half2_bits(hi[2], hi[3]), half2_bits(hi[4], hi[5]),
-                                  half2_bits(hi[6], hi[7]));
-      const uint4 L4 = make_uint4(half2_bits(lo[0], lo[1]), half2_bits(lo[2], lo[3]), half2_bits(lo[4], lo[5]),
-                                  half2_bits(lo[6], lo[7]));
-      *reinterpret_cast<uint4*>(frow + c) = H4;
-      if (f32) {
-        *reinterpret_cast<uint4*>(frow + F + c) = H4;
-        *reinterpret_cast<uint4*>(frow + 2 * F + c) = L4;
-      } else {
-        *reinterpret_cast<uint4*>(frow + F + c) = L4;
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        frow[c + t] = hi[t];
-        if (f32) { frow[F + c + t] = hi[t]; frow[2 * F + c + t] = lo[t]; }
-        else     { frow[F + c + t] = lo[t]; }
-      }
-    }
+    for (int t = 0; t < 8; ++t) w[t] = v[k0 + t];
+    put8(frow, F, f32, col + k0, 8, w);
   }
 }
 
@@ -165,26 +147,28 @@ __device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col,
 // its length sqrt(|local|^2 + eps); pair block; all zero for an empty
 // neighbourhood.  orow = this row's O accumulator divided by l (staged in
 // shared memory); (Gx,Gy,Gz) = sum_j a_ij o_G(j), the group-origin part of
-// the aggregated value points.  Also writes local_points.
-__device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, float* orow, float Gx, float Gy,
-                               float Gz, bool with_pair, const float (&R)[9], const float (&t)[3]) {
+// the aggregated value points.  fblk = the (residue, head) block of the
+// projection operand, lp = the residue's local points of this head [Q][3].
+__device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* orow, float Gx, float Gy,
+                               float Gz, bool with_pair, const float (&R)[9], const float (&t)[3], __half* fblk,
+                               float* lp) {
   const Plan& p = a.p;
-  const int H = p.H, Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.F;
-  __half* frow = a.feat + bi * p.Kgp;
-  float* lp = a.local_points + (bi * H + h) * (size_t)Q * 3;
-  if (h == 0)
-    for (int c = p.Kg; c < p.Kgp; ++c) frow[c] = __float2half_rn(0.f);
-  const int sc = h * Dv, xc = H * Dv + h * Q, pc = H * Dv + 4 * H * Q + h * Cz;
+  const int Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.Wh8;
+  const int sc = 0, xc = Dv, pc = Dv + 4 * Q;
+  auto zero = [](int) { return 0.f; };
+  if (p.Wh8 > p.Wh) put_run(fblk, F, p.f32, p.Wh, p.Wh8 - p.Wh, zero);
   if (empty) {
-    auto zero = [](int) { return 0.f; };
-    put_run(frow, F, p.f32, sc, Dv, zero);
-    for (int blk = 0; blk < 4; ++blk) put_run(frow, F, p.f32, xc + blk * H * Q, Q, zero);
-    if (with_pair) put_run(frow, F, p.f32, pc, Cz, zero);
-    for (int e = 0; e < 3 * Q; ++e) lp[e] = 0.f;
+    put_run(fblk, F, p.f32, sc, Dv + 4 * Q, zero);
+    if (with_pair) put_run(fblk, F, p.f32, pc, Cz, zero);
+    if (((3 * Q) & 3) == 0 && (reinterpret_cast<uintptr_t>(lp) & 15) == 0) {
+      for (int e = 0; e < 3 * Q; e += 4) *reinterpret_cast<float4*>(lp + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      for (int e = 0; e < 3 * Q; ++e) lp[e] = 0.f;
+    }
     return;
   }
   // scalar block
-  put_run(frow, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
+  put_run(fblk, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
   // points: aggregate (hi + lo halves + group-origin part), back into the query
   // frame; the local coordinates overwrite the consumed hi slots, the lengths the lo slots
   const int gofs = p.nsv * p.Dv8;
@@ -199,15 +183,22 @@ __device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, 
     orow[gofs + 3 * q + 1] = ly;
     orow[gofs + 3 * q + 2] = lz;
     orow[gofs + p.Q38 + q] = sqrtf(lx * lx + ly * ly + lz * lz + a.eps);
-    lp[3 * q + 0] = lx; lp[3 * q + 1] = ly; lp[3 * q + 2] = lz;
+  }
+  // local points [Q][3]: 16-byte stores where the row allows
+  if (((3 * Q) & 3) == 0 && (reinterpret_cast<uintptr_t>(lp) & 15) == 0) {
+    for (int e = 0; e < 3 * Q; e += 4)
+      *reinterpret_cast<float4*>(lp + e) =
+          make_float4(orow[gofs + e], orow[gofs + e + 1], orow[gofs + e + 2], orow[gofs + e + 3]);
+  } else {
+    for (int e = 0; e < 3 * Q; ++e) lp[e] = orow[gofs + e];
   }
   for (int x = 0; x < 3; ++x)
-    put_run(frow, F, p.f32, xc + x * H * Q, Q, [&](int q) { return orow[gofs + 3 * q + x]; });
-  put_run(frow, F, p.f32, xc + 3 * H * Q, Q, [&](int q) { return orow[gofs + p.Q38 + q]; });
+    put_run(fblk, F, p.f32, xc + x * Q, Q, [&](int q) { return orow[gofs + 3 * q + x]; });
+  put_run(fblk, F, p.f32, xc + 3 * Q, Q, [&](int q) { return orow[gofs + p.Q38 + q]; });
   // pair block through the factors (the tensor-memory path writes it otherwise)
   if (!with_pair) return;
   const int RCz = p.R * Cz;
-  put_run(frow, F, p.f32, pc, Cz, [&](int c) {
+  put_run(fblk, F, p.f32, pc, Cz, [&](int c) {
     float acc = 0.f;
     for (int rr = 0; rr < p.R; ++rr) {
       float u = orow[p.VHp + rr * Cz + c];
@@ -216,6 +207,35 @@ __device__ void write_features(const CoreArgs& a, size_t bi, int h, bool empty, 
     }
     return acc;
   });
+}
+
+// Shared-memory use of the feature epilogue, in the Qhat + ring memory:
+//   [0]      z1 rows of the query tile [128][R*Cz] (+16 bytes per row), copied
+//            during the last key tile, so they sit inside the Qhat buffer
+//            (dead once the last QK^T product has completed);
+//   [o_off]  O / l of each row, value-head columns [128][staged + 1] fp32.
+// z1 is prefetched only where both fit; otherwise the epilogue reads it from
+// global memory.
+struct EpiLayout {
+  bool fast_pair;   // pair block straight from TMEM (Cz a multiple of 32, z1 16-byte aligned)
+  bool z1_smem;     // z1 rows prefetched into shared memory
+  int staged;       // O columns staged per row
+  uint32_t z1_row_bytes, z1_stride, o_off;
+};
+
+__device__ __forceinline__ EpiLayout epi_layout(const Plan& p, const void* z1) {
+  EpiLayout e;
+  const uint32_t ring_end = (uint32_t)(p.nQc + p.nst) * kChunkBytes;
+  e.fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(z1) & 15) == 0;
+  e.staged = e.fast_pair ? p.VHp : p.Ocols;
+  e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.f32 ? 4 : 2));
+  e.z1_stride = e.z1_row_bytes + 16;
+  const uint32_t o_bytes = (uint32_t)kTile * (e.staged + 1) * 4;
+  e.z1_smem = e.fast_pair && (e.z1_row_bytes & 15) == 0 &&
+              (uint32_t)kTile * e.z1_stride <= (uint32_t)p.nQc * kChunkBytes;
+  e.o_off = e.z1_smem ? ((uint32_t)kTile * e.z1_stride + 1023u) & ~1023u : 0u;
+  if (e.o_off + o_bytes > ring_end) { e.z1_smem = false; e.o_off = 0; }
+  return e;
 }
 
 // Bounded wait that ignores the abort flag (used only to drain in-flight work).
@@ -308,14 +328,6 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float rowM = -INFINITY, rowL = 0.f, rowW[3] = {0.f, 0.f, 0.f};
   bool row_ok = false;
   float rowR[9], rowT[3];   // frame of the row's residue, loaded during the last tile
-  // z1 rows of the query tile, prefetched into the dead Qhat buffer once the
-  // last logit tile has been read (row stride padded by 16 bytes)
-  const size_t z1_row_bytes = (size_t)p.R * p.Cz * (p.f32 ? 4 : 2);
-  const size_t z1_stride = z1_row_bytes + 16;
-  const size_t z1_off = ((size_t)kTile * (p.VHp + 1) * 4 + 1023) & ~(size_t)1023;
-  const bool fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(a.z1) & 15) == 0;
-  const bool z1_smem = fast_pair && (z1_row_bytes & 15) == 0 &&
-                       z1_off + kTile * z1_stride <= (size_t)p.nQc * kChunkBytes;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -686,10 +698,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       for (int e = 0; e < 9; ++e) rowR[e] = ld_any(a.rot, bi * 9 + e, p.f32);
 #pragma unroll
       for (int e = 0; e < 3; ++e) rowT[e] = ld_any(a.trans, bi * 3 + e, p.f32);
-      if (z1_smem && i < N) {
-        const uint8_t* src = static_cast<const uint8_t*>(a.z1) + bi * z1_row_bytes;
-        uint8_t* dst = smem + z1_off + (size_t)(wq * 32 + lane) * z1_stride;
-        for (size_t o = 0; o < z1_row_bytes; o += 16) cp_async16(dst + o, src + o);
+      const EpiLayout el = epi_layout(p, a.z1);
+      if (el.z1_smem && i < N) {
+        const uint8_t* src = static_cast<const uint8_t*>(a.z1) + bi * el.z1_row_bytes;
+        uint8_t* dst = smem + (size_t)(wq * 32 + lane) * el.z1_stride;
+        for (uint32_t o = 0; o < el.z1_row_bytes; o += 16) cp_async16(dst + o, src + o);
       }
       cp_async_commit();
     }
@@ -713,14 +726,16 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   ttr.ev(42);
+  const EpiLayout el = epi_layout(p, a.z1);
+  const bool fast_pair = el.fast_pair;
   if (warp >= 4 && *abort_flag == 0) {
     const int wq = warp - 4;
     const int r = wq * 32 + lane;
     const int i = qt * kTile + r;
     const bool in_range = i < N;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
-    const int staged = fast_pair ? p.VHp : p.Ocols;         // columns staged in shared memory
-    float* orow = reinterpret_cast<float*>(smem) + (size_t)r * (staged + 1);
+    const int staged = el.staged;                           // columns staged in shared memory
+    float* orow = reinterpret_cast<float*>(smem + el.o_off) + (size_t)r * (staged + 1);
     const float inv = rowL > 0.f ? 1.f / rowL : 0.f;
     const bool live = row_ok && nkt > 0;
     if (live) {
@@ -735,6 +750,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     ttr.ev(45);
     const size_t bi = (size_t)b * N + (in_range ? i : 0);
     const bool empty = !(rowL > 0.f) || !live;
+    // this row's head block of the projection operand and its local points
+    __half* fblk = a.feat + bi * p.Kgp + (size_t)h * p.nseg * p.Wh8;
+    float* lp = a.local_points + (bi * p.H + h) * (size_t)p.Q * 3;
     if (in_range) {
       a.stats[(size_t)bh * N + i] = make_float2(rowM, rowL);
       if (a.lse != nullptr) {
@@ -742,15 +760,18 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         a.lse[(size_t)bh * N + i] = rowL > 0.f ? (rowM + log2f(rowL)) * kLn2 + qv.w : -INFINITY;
       }
       if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
-      write_features(a, bi, h, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT);
+      if (h == 0)
+        for (int c = p.Kg; c < p.Kgp; ++c) a.feat[bi * p.Kgp + c] = __float2half_rn(0.f);
+      write_features(a, bi, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT,
+                     fblk, lp);
     }
     ttr.ev(46);
     if (fast_pair) {
       // pair block straight from tensor memory, 32 channels at a time
-      const int Cz = p.Cz, RCz = p.R * Cz, pcol = p.H * p.Dv + 4 * p.H * p.Q + h * Cz;
-      __half* frow = a.feat + bi * p.Kgp;
+      const int Cz = p.Cz, RCz = p.R * Cz, pcol = p.Dv + 4 * p.Q;
+      __half* frow = fblk;
       cp_async_wait_all();
-      const uint8_t* zs = smem + z1_off + (size_t)r * z1_stride;
+      const uint8_t* zs = smem + (size_t)r * el.z1_stride;
       for (int c0 = 0; c0 < Cz; c0 += 32) {
         float acc[32];
 #pragma unroll
@@ -773,19 +794,19 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const size_t zrel = (size_t)rr * Cz + c0;
             float zv[32];
             if (p.f32) {
-              const float4* z4 = z1_smem ? reinterpret_cast<const float4*>(zs) + zrel / 4
+              const float4* z4 = el.z1_smem ? reinterpret_cast<const float4*>(zs) + zrel / 4
                                          : reinterpret_cast<const float4*>(static_cast<const float*>(a.z1) + zoff);
 #pragma unroll
               for (int k = 0; k < 8; ++k) {
-                const float4 t4 = z1_smem ? z4[k] : __ldg(z4 + k);
+                const float4 t4 = el.z1_smem ? z4[k] : __ldg(z4 + k);
                 zv[4 * k] = t4.x; zv[4 * k + 1] = t4.y; zv[4 * k + 2] = t4.z; zv[4 * k + 3] = t4.w;
               }
             } else {
-              const uint4* z4 = z1_smem ? reinterpret_cast<const uint4*>(zs) + zrel / 8
+              const uint4* z4 = el.z1_smem ? reinterpret_cast<const uint4*>(zs) + zrel / 8
                                         : reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.z1) + zoff);
 #pragma unroll
               for (int k = 0; k < 4; ++k) {
-                const uint4 t4 = z1_smem ? z4[k] : __ldg(z4 + k);
+                const uint4 t4 = el.z1_smem ? z4[k] : __ldg(z4 + k);
                 const uint32_t w4[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
@@ -798,12 +819,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv, acc[e]);
           }
         }
-        if (in_range) put_run32(frow, p.F, p.f32, pcol + c0, acc);
+        if (in_range) put_run32(frow, p.Wh8, p.f32, pcol + c0, acc);
       }
     }
     ttr.ev(47);
   }
-
   // ---------------------------------------------------------------- teardown
   ttr.ev(43);
   tc_fence_before();

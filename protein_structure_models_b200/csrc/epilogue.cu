@@ -13,10 +13,29 @@
 namespace fipa {
 namespace {
 
-// w_out [F, Cout] -> wT [Cout_pad, Kgp] fp16, K-major, matching the feature parts:
+// w_out [F, Cout] -> wT [Cout_pad, Kgp] fp16, K-major, in the head-block order
+// of the projection operand (plan.h): column k = (h * nseg + seg) * Wh8 + j
+// holds row f(h, j) of w_out, f the page's head-major feature index:
+//   j <  Dv           scalar   f = h*Dv + j
+//   j <  Dv + 4Q      x,y,z,len  f = H*Dv + blk*H*Q + h*Q + q   (j = Dv + blk*Q + q)
+//   j <  Dv + 4Q + Cz pair     f = H*Dv + 4*H*Q + h*Cz + c
+// and zero for the padding j >= Wh and k >= Kg.  Segments:
 //   bf16 inputs: [ w | w ]            (w is exact in fp16)
 //   f32  inputs: [ w hi | w lo | w hi ]
-// 32 x 32 tiles transposed through shared memory (coalesced reads and writes).
+// 32 x 32 tiles over (f, n) transposed through shared memory (coalesced reads).
+__device__ __forceinline__ int feature_block_col(const Plan& p, int f, int* h) {
+  const int HDv = p.H * p.Dv, HQ = p.H * p.Q;
+  if (f < HDv) { *h = f / p.Dv; return f - *h * p.Dv; }
+  if (f < HDv + 4 * HQ) {
+    const int g = f - HDv, blk = g / HQ, rem = g - blk * HQ;
+    *h = rem / p.Q;
+    return p.Dv + blk * p.Q + (rem - *h * p.Q);
+  }
+  const int g = f - HDv - 4 * HQ;
+  *h = g / p.Cz;
+  return p.Dv + 4 * p.Q + (g - *h * p.Cz);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) fipa_weight_prep_kernel(const Plan p, const T* w, __half* wT, int cout_pad) {
   __shared__ float tile[32][33];
@@ -27,29 +46,61 @@ __global__ void __launch_bounds__(256) fipa_weight_prep_kernel(const Plan p, con
     tile[k][tx] = (f < p.F && n < p.Cout) ? ld_in(w, (size_t)f * p.Cout + n) : 0.f;
   }
   __syncthreads();
-  const int nseg = p.f32 ? 3 : 2;
+  const int f = f0 + tx;
+  int h = 0;
+  const int j = f < p.F ? feature_block_col(p, f, &h) : 0;
   for (int k = ty; k < 32; k += 8) {
-    const int n = n0 + k, f = f0 + tx;
+    const int n = n0 + k;
     if (n >= cout_pad || f >= p.F) continue;
     const float v = tile[tx][k];
     const __half hi = __float2half_rn(v), lo = __float2half_rn(v - __half2float(hi));
-    for (int seg = 0; seg < nseg; ++seg) wT[(size_t)n * p.Kgp + seg * p.F + f] = (p.f32 && seg == 1) ? lo : hi;
+    __half* row = wT + (size_t)n * p.Kgp + (size_t)h * p.nseg * p.Wh8 + j;
+    for (int seg = 0; seg < p.nseg; ++seg) row[seg * p.Wh8] = (p.f32 && seg == 1) ? lo : hi;
   }
   if (blockIdx.x == 0) {
+    // padding columns: j in [Wh, Wh8) of every head segment, and [Kg, Kgp)
+    const int padw = p.Wh8 - p.Wh, nblk = p.H * p.nseg;
     for (int k = ty; k < 32; k += 8) {
       const int n = n0 + k;
-      if (n < cout_pad)
-        for (int c = p.Kg + tx; c < p.Kgp; c += 32) wT[(size_t)n * p.Kgp + c] = __float2half_rn(0.f);
+      if (n >= cout_pad) continue;
+      __half* row = wT + (size_t)n * p.Kgp;
+      for (int e = tx; e < nblk * padw; e += 32) {
+        const int bk = e / padw;
+        row[(size_t)bk * p.Wh8 + p.Wh + (e - bk * padw)] = __float2half_rn(0.f);
+      }
+      for (int c = p.Kg + tx; c < p.Kgp; c += 32) row[c] = __float2half_rn(0.f);
     }
   }
 }
 
-// Sum of the split-K partials, + b_out, zero for an empty neighbourhood.
+// Sum of the split-K partials in split order (deterministic), + b_out, zero
+// for an empty neighbourhood; 4 outputs per thread where Cout allows.
 template <typename T>
 __global__ void fipa_proj_reduce_kernel(const Plan p, const float* part, const T* b_out, const uint8_t* rowflag,
                                         float* update) {
   const int cpad = rup(p.Cout, p.ntile_out);
-  const size_t total = (size_t)p.B * p.N * p.Cout, plane = (size_t)p.B * p.N * cpad;
+  const size_t M = (size_t)p.B * p.N, plane = M * cpad;
+  const bool vec = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(update) & 15) == 0;
+  if (vec) {
+    const int cq = p.Cout / 4;
+    const size_t total = M * cq;
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+      const size_t m = e / cq;
+      const int n = (int)(e - m * cq) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int z = 0; z < p.gemm_ks; ++z) {
+        const float4 v = *reinterpret_cast<const float4*>(part + z * plane + m * cpad + n);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const bool keep = rowflag[m] != 0;
+      reinterpret_cast<float4*>(update)[e] =
+          keep ? make_float4(acc.x + ld_in(b_out, n), acc.y + ld_in(b_out, n + 1), acc.z + ld_in(b_out, n + 2),
+                             acc.w + ld_in(b_out, n + 3))
+               : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    return;
+  }
+  const size_t total = M * p.Cout;
   for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
     const size_t m = e / p.Cout;
     const int n = (int)(e - m * p.Cout);
@@ -153,35 +204,68 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(acc_full, 0) && global_timer_ns() - t0 < a.timeout_ns) {}
     }
-  } else if (warp >= 4) {
-    const int wq = warp - 4;
-    const int m = m0 + wq * 32 + lane;
-    bool ok = mbar_wait(acc_full, 0, wc, 23);
-    ok = __all_sync(0xffffffffu, ok) && !*abort_flag;
-    tc_fence_after();
-    if (ok) {
-      const bool live = m < p.B * p.N;
-      const bool keep = live && a.rowflag[m] != 0;
-      const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
-      const int cpad = rup(p.Cout, ntile);
-      float* prow = a.part + ((size_t)blockIdx.z * p.B * p.N + (size_t)m) * cpad;
-      for (int c = 0; c < ntile; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(trow + (uint32_t)c, o);
-        tmem_ld_wait();
-        if (live && p.gemm_ks > 1) {
+  }
+
+  // ---- epilogue, all 8 warps: the accumulator goes TMEM -> registers ->
+  // a staged tile in the (now idle) pipeline memory, [128][ntile + 4] fp32,
+  // then out as whole rows with 16-byte stores (warps w and w+4 read the same
+  // TMEM lanes and split the 32-column chunks)
+  bool ok = mbar_wait(acc_full, 0, wc, 23);
+  ok = __syncthreads_and(ok && *abort_flag == 0) != 0;
+  tc_fence_after();
+  const int sstride = ntile + 4;
+  float* stile = reinterpret_cast<float*>(smem);
+  if (ok) {
+    const int q4 = warp & 3, half = warp >> 2;
+    const int r = q4 * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(q4 * 32) << 16);
+    float* srow = stile + (size_t)r * sstride;
+    for (int c = half * 32; c < ntile; c += 64) {
+      uint32_t o[32];
+      tmem_ld32(trow + (uint32_t)c, o);
+      tmem_ld_wait();
+      if (c + 32 <= ntile) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) prow[n0 + c + e] = __uint_as_float(o[e]);
-        } else if (live) {
-          float* urow = a.update + (size_t)m * p.Cout;
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(srow + c + e) = make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
+                                                                 __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int n = n0 + c + e;
-            if (n < p.Cout) {
-              const float bo = p.f32 ? static_cast<const float*>(a.b_out)[n]
-                                     : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n]);
-              urow[n] = keep ? __uint_as_float(o[e]) + bo : 0.f;
-            }
+        for (int e = 0; e < 32; ++e)
+          if (c + e < ntile) srow[c + e] = __uint_as_float(o[e]);
+      }
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    const int M = p.B * p.N, cpad = rup(p.Cout, ntile), nq = ntile / 4;
+    const bool vec_out = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(a.update) & 15) == 0;
+    for (int rr = warp; rr < kTile; rr += 8) {
+      const int m = m0 + rr;
+      if (m >= M) break;
+      const float* srow = stile + (size_t)rr * sstride;
+      if (p.gemm_ks > 1) {
+        float4* prow = reinterpret_cast<float4*>(a.part + ((size_t)blockIdx.z * M + m) * cpad + n0);
+        for (int c4 = lane; c4 < nq; c4 += 32) prow[c4] = *reinterpret_cast<const float4*>(srow + 4 * c4);
+      } else {
+        const bool keep = a.rowflag[m] != 0;
+        float* urow = a.update + (size_t)m * p.Cout;
+        for (int c4 = lane; c4 < nq; c4 += 32) {
+          const int n = n0 + 4 * c4;
+          const float4 v = *reinterpret_cast<const float4*>(srow + 4 * c4);
+          float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float bo = n + e < p.Cout ? (p.f32 ? static_cast<const float*>(a.b_out)[n + e]
+                                                    : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n + e]))
+                                            : 0.f;
+            w[e] = keep ? w[e] + bo : 0.f;
+          }
+          if (vec_out && n + 4 <= p.Cout) {
+            *reinterpret_cast<float4*>(urow + n) = make_float4(w[0], w[1], w[2], w[3]);
+          } else {
+            for (int e = 0; e < 4; ++e)
+              if (n + e < p.Cout) urow[n + e] = w[e];
           }
         }
       }

@@ -94,7 +94,13 @@ struct Plan {
   FastDiv fd_H, fd_P, fd_Q, fd_Cz;               // divisors of the lift kernel's index maps
   FastDiv fd_nQ8, fd_nK8, fd_nV8, fd_nZ8;        // 16-byte chunks per lifted row type
   FastDiv fd_D8v, fd_Dv8v, fd_RC8v;              // 8-value vectors per staged row
-  int Kg, Kgp;        // output-projection K (2F or 3F) and padded
+  // Output-projection operand: one block per head, in head order, each block
+  // nseg segments (bf16: [hi | lo], f32: [hi | hi | lo]) of Wh8 columns holding
+  // [scalar (Dv) | x (Q) | y (Q) | z (Q) | lengths (Q) | pair (Cz) | pad].  The
+  // projection's sum over k is taken in this order; the weights are permuted
+  // to match, so the result is features @ w_out in the page's feature order.
+  int Wh, Wh8, nseg;  // head-block feature width, padded to 8, segments
+  int Kg, Kgp;        // output-projection K (H * nseg * Wh8) and padded
   int ntile_out;      // output-projection N tile (<= 256)
   int gemm_ks;        // output-projection split-K factor
   int gemm_nks;       // K chunks per split
@@ -181,14 +187,17 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.fd_D8v = make_fastdiv(p.D8 / 8); p.fd_Dv8v = make_fastdiv(p.Dv8 / 8); p.fd_RC8v = make_fastdiv(p.RC8 / 8);
   if (p.lift_smem > 160 * 1024) { *why = "prologue staging exceeds shared memory (H*Cz or R*Cz too large)"; return 2; }
   // output projection
-  p.Kg = (f32 ? 3 : 2) * p.F;
+  p.Wh = Dv + 4 * Q + Cz;
+  p.Wh8 = rup(p.Wh, 8);
+  p.nseg = f32 ? 3 : 2;
+  p.Kg = H * p.nseg * p.Wh8;
   p.Kgp = rup(p.Kg, kChunk);
   // N tile and split-K so that the grid covers the SMs (deterministic split-K:
   // partial sums go to the workspace and a reduce kernel adds them in order)
   {
+    // N tile = all of Cout up to 256 (wide MMAs); split-K fills the SMs
     const int mt = cdiv(B * N, kTile), nk = p.Kgp / kChunk;
-    int nt_w = Cout >= 256 ? 256 : rup(Cout, 16);
-    while (mt * cdiv(Cout, nt_w) < 148 && nt_w > 64) nt_w = rup(nt_w / 2, 16);
+    const int nt_w = Cout >= 256 ? 256 : rup(Cout, 16);
     p.ntile_out = nt_w;
     const int tiles = mt * cdiv(Cout, nt_w);
     int ks = tiles >= 148 ? 1 : cdiv(148, tiles);
