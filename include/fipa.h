@@ -173,7 +173,9 @@ fipa_status fipa_sync_status(fipa_handle* h, void* stream);
 /* Profiling aid (stage timing).  With `enable` nonzero, later fipa_forward
  * calls on this handle record a CUDA event before and after each of their
  * kernels on the call's stream; the events are created here, so fipa_forward
- * still allocates nothing.  `enable` = 0 turns recording off and frees them. */
+ * still allocates nothing.  `enable` = 0 turns recording off and frees them.
+ * A CUDA graph captured from a timed call records into these events on every
+ * replay: release such a graph before turning timing off. */
 fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable);
 
 /* Device time in milliseconds of each stage of the most recent fipa_forward
