@@ -179,11 +179,13 @@ fipa_status fipa_sync_status(fipa_handle* h, void* stream);
 fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable);
 
 /* Device time in milliseconds of each stage of the most recent fipa_forward
- * recorded with stage timing on, in launch order: [0] prologue (tile origins
- * and lifted rows), [1] fused attention core with the feature epilogue,
- * [2] output-weight preparation, [3] output projection, [4] attention output
- * (0 when not requested).  Waits for that call's last event.  `n` = capacity
- * of `ms` (up to 5 values are written). */
+ * recorded with stage timing on, in launch order: [0] prologue (output-weight
+ * preparation, group origins and lifted rows), [1] fused attention core with
+ * the feature epilogue, [2] output projection, [3] attention output (0 when
+ * not requested).  Each interval spans one kernel launch between two event
+ * records.  Waits for that call's last event.  `n` = capacity of `ms` (up to
+ * FIPA_STAGES values are written). */
+#define FIPA_STAGES 4
 fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n);
 
 /* Debug tracing.  When the environment variable FIPA_TRACE_CTA=<n> is set at

@@ -7,108 +7,16 @@
 //   each flattened head-major; update = features @ w_out + b_out, zero when empty.
 // The pair aggregate is rebuilt from the factors: sum_j a_ij z_ij[c] =
 // sum_r z1[i,r,c] U[r,c] with U = sum_j a_ij z2[j,r,c] from the core.
+#include <cooperative_groups.h>
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
 namespace fipa {
 namespace {
 
-// w_out [F, Cout] -> wT [Cout_pad, Kgp] fp16, K-major, in the head-block order
-// of the projection operand (plan.h): column k = (h * nseg + seg) * Wh8 + j
-// holds row f(h, j) of w_out, f the page's head-major feature index:
-//   j <  Dv           scalar   f = h*Dv + j
-//   j <  Dv + 4Q      x,y,z,len  f = H*Dv + blk*H*Q + h*Q + q   (j = Dv + blk*Q + q)
-//   j <  Dv + 4Q + Cz pair     f = H*Dv + 4*H*Q + h*Cz + c
-// and zero for the padding j >= Wh and k >= Kg.  Segments:
-//   bf16 inputs: [ w | w ]            (w is exact in fp16)
-//   f32  inputs: [ w hi | w lo | w hi ]
-// 32 x 32 tiles over (f, n) transposed through shared memory (coalesced reads).
-__device__ __forceinline__ int feature_block_col(const Plan& p, int f, int* h) {
-  const int HDv = p.H * p.Dv, HQ = p.H * p.Q;
-  if (f < HDv) { *h = f / p.Dv; return f - *h * p.Dv; }
-  if (f < HDv + 4 * HQ) {
-    const int g = f - HDv, blk = g / HQ, rem = g - blk * HQ;
-    *h = rem / p.Q;
-    return p.Dv + blk * p.Q + (rem - *h * p.Q);
-  }
-  const int g = f - HDv - 4 * HQ;
-  *h = g / p.Cz;
-  return p.Dv + 4 * p.Q + (g - *h * p.Cz);
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256) fipa_weight_prep_kernel(const Plan p, const T* w, __half* wT, int cout_pad) {
-  __shared__ float tile[32][33];
-  const int f0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  for (int k = ty; k < 32; k += 8) {
-    const int f = f0 + k, n = n0 + tx;
-    tile[k][tx] = (f < p.F && n < p.Cout) ? ld_in(w, (size_t)f * p.Cout + n) : 0.f;
-  }
-  __syncthreads();
-  const int f = f0 + tx;
-  int h = 0;
-  const int j = f < p.F ? feature_block_col(p, f, &h) : 0;
-  for (int k = ty; k < 32; k += 8) {
-    const int n = n0 + k;
-    if (n >= cout_pad || f >= p.F) continue;
-    const float v = tile[tx][k];
-    const __half hi = __float2half_rn(v), lo = __float2half_rn(v - __half2float(hi));
-    __half* row = wT + (size_t)n * p.Kgp + (size_t)h * p.nseg * p.Wh8 + j;
-    for (int seg = 0; seg < p.nseg; ++seg) row[seg * p.Wh8] = (p.f32 && seg == 1) ? lo : hi;
-  }
-  if (blockIdx.x == 0) {
-    // padding columns: j in [Wh, Wh8) of every head segment, and [Kg, Kgp)
-    const int padw = p.Wh8 - p.Wh, nblk = p.H * p.nseg;
-    for (int k = ty; k < 32; k += 8) {
-      const int n = n0 + k;
-      if (n >= cout_pad) continue;
-      __half* row = wT + (size_t)n * p.Kgp;
-      for (int e = tx; e < nblk * padw; e += 32) {
-        const int bk = e / padw;
-        row[(size_t)bk * p.Wh8 + p.Wh + (e - bk * padw)] = __float2half_rn(0.f);
-      }
-      for (int c = p.Kg + tx; c < p.Kgp; c += 32) row[c] = __float2half_rn(0.f);
-    }
-  }
-}
-
-// Sum of the split-K partials in split order (deterministic), + b_out, zero
-// for an empty neighbourhood; 4 outputs per thread where Cout allows.
-template <typename T>
-__global__ void fipa_proj_reduce_kernel(const Plan p, const float* part, const T* b_out, const uint8_t* rowflag,
-                                        float* update) {
-  const int cpad = rup(p.Cout, p.ntile_out);
-  const size_t M = (size_t)p.B * p.N, plane = M * cpad;
-  const bool vec = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(update) & 15) == 0;
-  if (vec) {
-    const int cq = p.Cout / 4;
-    const size_t total = M * cq;
-    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-      const size_t m = e / cq;
-      const int n = (int)(e - m * cq) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int z = 0; z < p.gemm_ks; ++z) {
-        const float4 v = *reinterpret_cast<const float4*>(part + z * plane + m * cpad + n);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      const bool keep = rowflag[m] != 0;
-      reinterpret_cast<float4*>(update)[e] =
-          keep ? make_float4(acc.x + ld_in(b_out, n), acc.y + ld_in(b_out, n + 1), acc.z + ld_in(b_out, n + 2),
-                             acc.w + ld_in(b_out, n + 3))
-               : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    return;
-  }
-  const size_t total = M * p.Cout;
-  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const size_t m = e / p.Cout;
-    const int n = (int)(e - m * p.Cout);
-    float acc = 0.f;
-    for (int z = 0; z < p.gemm_ks; ++z) acc += part[z * plane + m * cpad + n];
-    update[e] = rowflag[m] ? acc + ld_in(b_out, n) : 0.f;
-  }
-}
+namespace cg = cooperative_groups;
 
 // ------------------------------------------------------------------ projection GEMM
 struct ProjArgs {
@@ -116,9 +24,10 @@ struct ProjArgs {
   const void* b_out;
   const uint8_t* rowflag;
   float* update;
-  float* part;
   int* status;
   unsigned long long timeout_ns;
+  long long* trace;   // debug timeline of one CTA (last slots of the MMA role's log), or null
+  int trace_cta;
 };
 
 // update[m, n] = sum_k feat[m, k] wT[n, k] + b_out[n], zero for empty rows.
@@ -141,6 +50,10 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   int* abort_flag = reinterpret_cast<int*>(tail + 260);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kTile, n0 = blockIdx.y * ntile;
+  const bool timeline = a.trace != nullptr && threadIdx.x == 0 &&
+                        (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) == a.trace_cta;
+  Tracer ttr{timeline ? a.trace + (size_t)1 * 2 * kTraceCap : nullptr, kTraceCap - 8};
+  ttr.ev(50);
   const int nk_all = p.Kgp / kChunk;
   const int k0 = blockIdx.z * p.gemm_nks;
   const int nk = min(nk_all, k0 + p.gemm_nks) - k0;      // K chunks of this split
@@ -158,6 +71,7 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const WaitCtx wc{abort_flag, a.status, a.timeout_ns};
+  ttr.ev(51);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -210,7 +124,9 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   // a staged tile in the (now idle) pipeline memory, [128][ntile + 4] fp32,
   // then out as whole rows with 16-byte stores (warps w and w+4 read the same
   // TMEM lanes and split the 32-column chunks)
+  ttr.ev(52);
   bool ok = mbar_wait(acc_full, 0, wc, 23);
+  ttr.ev(53);
   ok = __syncthreads_and(ok && *abort_flag == 0) != 0;
   tc_fence_after();
   const int sstride = ntile + 4;
@@ -236,41 +152,61 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
       }
     }
   }
-  __syncthreads();
+  // split-K across the cluster (grid z = cluster z = gemm_ks): every CTA has
+  // staged its partial tile; CTA z then sums rows [z*R, (z+1)*R) of all the
+  // cluster's tiles, in split order (deterministic), through distributed
+  // shared memory, and writes them.  The second cluster barrier keeps every
+  // tile alive until its readers are done.
+  const int ks = p.gemm_ks;
+  cg::cluster_group cluster = cg::this_cluster();
+  if (ks > 1) cluster.sync();
+  else __syncthreads();
+  ttr.ev(54);
   if (ok) {
-    const int M = p.B * p.N, cpad = rup(p.Cout, ntile), nq = ntile / 4;
+    const int M = p.B * p.N, nq = ntile / 4;
     const bool vec_out = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(a.update) & 15) == 0;
-    for (int rr = warp; rr < kTile; rr += 8) {
+    const int rows = (kTile + ks - 1) / ks, r0 = (int)blockIdx.z * rows, r1 = min(kTile, r0 + rows);
+    for (int rr = r0 + warp; rr < r1; rr += 8) {
       const int m = m0 + rr;
       if (m >= M) break;
-      const float* srow = stile + (size_t)rr * sstride;
-      if (p.gemm_ks > 1) {
-        float4* prow = reinterpret_cast<float4*>(a.part + ((size_t)blockIdx.z * M + m) * cpad + n0);
-        for (int c4 = lane; c4 < nq; c4 += 32) prow[c4] = *reinterpret_cast<const float4*>(srow + 4 * c4);
-      } else {
-        const bool keep = a.rowflag[m] != 0;
-        float* urow = a.update + (size_t)m * p.Cout;
-        for (int c4 = lane; c4 < nq; c4 += 32) {
-          const int n = n0 + 4 * c4;
-          const float4 v = *reinterpret_cast<const float4*>(srow + 4 * c4);
-          float w[4] = {v.x, v.y, v.z, v.w};
+      const bool keep = a.rowflag[m] != 0;
+      float* urow = a.update + (size_t)m * p.Cout;
+      for (int c4 = lane; c4 < nq; c4 += 32) {
+        const int n = n0 + 4 * c4;
+        // all splits' loads in flight together, then added in split order
+        float4 t[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float bo = n + e < p.Cout ? (p.f32 ? static_cast<const float*>(a.b_out)[n + e]
-                                                    : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n + e]))
-                                            : 0.f;
-            w[e] = keep ? w[e] + bo : 0.f;
+        for (int z = 0; z < 8; ++z) {
+          if (z < ks) {
+            const float* tz = ks > 1 ? cluster.map_shared_rank(stile, z) : stile;
+            t[z] = *reinterpret_cast<const float4*>(tz + (size_t)rr * sstride + 4 * c4);
           }
-          if (vec_out && n + 4 <= p.Cout) {
-            *reinterpret_cast<float4*>(urow + n) = make_float4(w[0], w[1], w[2], w[3]);
-          } else {
-            for (int e = 0; e < 4; ++e)
-              if (n + e < p.Cout) urow[n + e] = w[e];
-          }
+        }
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int z = 0; z < 8; ++z) {
+          if (z < ks) { v.x += t[z].x; v.y += t[z].y; v.z += t[z].z; v.w += t[z].w; }
+        }
+        float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float bo = n + e < p.Cout ? (p.f32 ? static_cast<const float*>(a.b_out)[n + e]
+                                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n + e]))
+                                          : 0.f;
+          w[e] = keep ? w[e] + bo : 0.f;
+        }
+        if (vec_out && n + 4 <= p.Cout) {
+          *reinterpret_cast<float4*>(urow + n) = make_float4(w[0], w[1], w[2], w[3]);
+        } else {
+          for (int e = 0; e < 4; ++e)
+            if (n + e < p.Cout) urow[n + e] = w[e];
         }
       }
     }
   }
+  ttr.ev(55);
+  if (ks > 1) cluster.sync();
+  ttr.ev(56);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -282,37 +218,71 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
 }  // namespace
 
-cudaError_t launch_weight_prep(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s) {
-  const int cout_pad = rup(p.Cout, p.ntile_out);
-  dim3 grid((unsigned)cdiv(p.F, 32), (unsigned)cdiv(cout_pad, 32)), block(32, 8);
-  if (p.f32)
-    fipa_weight_prep_kernel<float><<<grid, block, 0, s>>>(p, static_cast<const float*>(in.w_out), w.wT, cout_pad);
-  else
-    fipa_weight_prep_kernel<__nv_bfloat16><<<grid, block, 0, s>>>(
-        p, static_cast<const __nv_bfloat16*>(in.w_out), w.wT, cout_pad);
-  return cudaGetLastError();
+// Largest split-K factor <= p.gemm_ks whose clusters (one per output tile, of
+// ks CTAs) are all resident at once, so no tile waits for a second wave; the
+// resident-cluster counts come from the occupancy API, once per device.
+static int resident_split(const Plan& p, int tiles) {
+  static std::mutex mu;
+  static int cached[64][9] = {};          // [device][ks] max active clusters (0 = unknown)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  const int nk = p.Kgp / kChunk;
+  for (int ks = p.gemm_ks; ks > 1; --ks) {
+    int n;
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      n = cached[dev][ks];
+    }
+    if (n == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(1, 1, ks);
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = p.gemm_smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 1;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = (unsigned)ks;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, fipa_out_proj_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = -1;
+      }
+      std::lock_guard<std::mutex> lock(mu);
+      cached[dev][ks] = n;
+    }
+    if (n > 0 && tiles <= n && cdiv(nk, ks) >= 4) return ks;
+  }
+  return 1;
 }
 
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl, cudaStream_t s) {
-  ProjArgs a{p, in.b_out, w.rowflag, out.update, w.part, ctl.status, ctl.timeout_ns};
+  ProjArgs a{p, in.b_out, w.rowflag, out.update, ctl.status, ctl.timeout_ns, ctl.trace, ctl.trace_cta};
   const size_t BN = (size_t)p.B * p.N;
-  dim3 grid((unsigned)((BN + kTile - 1) / kTile), (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out),
-            (unsigned)p.gemm_ks);
+  const unsigned mt = (unsigned)((BN + kTile - 1) / kTile), nt = (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out);
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_out_proj_kernel));
   if (e != cudaSuccess) return e;
-  fipa_out_proj_kernel<<<grid, 256, p.gemm_smem, s>>>(tmA, tmB, a);
-  if (p.gemm_ks > 1) {
-    const size_t total = BN * p.Cout;
-    unsigned g = (unsigned)((total + 255) / 256);
-    if (g > 148 * 16) g = 148 * 16;
-    if (p.f32)
-      fipa_proj_reduce_kernel<float><<<g, 256, 0, s>>>(p, w.part, static_cast<const float*>(in.b_out), w.rowflag,
-                                                         out.update);
-    else
-      fipa_proj_reduce_kernel<__nv_bfloat16><<<g, 256, 0, s>>>(
-          p, w.part, static_cast<const __nv_bfloat16*>(in.b_out), w.rowflag, out.update);
-  }
+  const int nk = p.Kgp / kChunk;
+  const int ks = p.gemm_ks > 1 ? resident_split(p, (int)(mt * nt)) : 1;
+  a.p.gemm_nks = cdiv(nk, ks);
+  a.p.gemm_ks = cdiv(nk, a.p.gemm_nks);
+  // the split-K CTAs of one output tile form a cluster along z
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mt, nt, (unsigned)a.p.gemm_ks);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = p.gemm_smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)a.p.gemm_ks;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fipa_out_proj_kernel, tmA, tmB, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -18,6 +18,9 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// stage-timing intervals: prologue, core, output projection, attention output
+constexpr int kStages = FIPA_STAGES;
+
 struct fipa_handle {
   int device = 0;
   fipa_dtype dtype = FIPA_BF16;
@@ -29,7 +32,7 @@ struct fipa_handle {
   std::string last_error;
   bool timing = false;
   bool timed_call = false;
-  cudaEvent_t ev[6] = {};
+  cudaEvent_t ev[kStages + 1] = {};
   long long* d_trace = nullptr;
   int trace_cta = -1;
   int pair_split = 1;
@@ -174,9 +177,9 @@ FIPA_API fipa_status fipa_stage_times(fipa_handle* h, float* ms, int n) {
   if (h == nullptr || ms == nullptr || n < 0) return FIPA_ERR_INVALID_ARG;
   if (!h->timing || !h->timed_call) return fail(h, FIPA_ERR_INVALID_ARG, "no timed fipa_forward call");
   DeviceGuard g(h->device);
-  cudaError_t e = cudaEventSynchronize(h->ev[5]);
+  cudaError_t e = cudaEventSynchronize(h->ev[kStages]);
   if (e != cudaSuccess) return cuda_fail(h, "event sync", e);
-  for (int k = 0; k < 5 && k < n; ++k) {
+  for (int k = 0; k < kStages && k < n; ++k) {
     float t = 0.f;
     e = cudaEventElapsedTime(&t, h->ev[k], h->ev[k + 1]);
     if (e != cudaSuccess) return cuda_fail(h, "event time", e);
@@ -229,8 +232,8 @@ FIPA_API fipa_status fipa_kernel_count(const fipa_handle* hc, const fipa_dims* d
   const int rc = plan_for(h, dims, p);
   if (rc == 1) return FIPA_ERR_INVALID_ARG;
   if (rc == 2) return FIPA_ERR_UNSUPPORTED;
-  // origin, lift, core, weight prep, projection (+ split-K reduce) (+ attention)
-  *count = 5 + (p.gemm_ks > 1 ? 1 : 0) + (with_attention ? 1 : 0);
+  // prologue (weight prep + lift), core, projection (+ attention)
+  *count = 3 + (with_attention ? 1 : 0);
   return FIPA_OK;
 }
 
@@ -307,7 +310,6 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
   w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
   w.rowflag = ws + p.off_rowflag;
-  w.part = reinterpret_cast<float*>(ws + p.off_part);
 
   fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
                   w_out, b_out, (float)eps};
@@ -343,16 +345,14 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   if ((e = fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s)) != cudaSuccess)
     return cuda_fail(h, "core launch", e);
   mark(2);
-  if ((e = fipa::launch_weight_prep(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "weight prep launch", e);
-  mark(3);
   if ((e = fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s)) != cudaSuccess)
     return cuda_fail(h, "output projection launch", e);
-  mark(4);
+  mark(3);
   if (out_attention != nullptr) {
     if ((e = fipa::launch_attention_dump(p, in, w, out, s)) != cudaSuccess)
       return cuda_fail(h, "attention launch", e);
   }
-  mark(5);
+  mark(4);
   h->timed_call = rec;
   return FIPA_OK;
 }

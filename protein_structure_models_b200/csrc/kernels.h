@@ -58,7 +58,6 @@ struct Work {
   __half *feat;    // [B*N, Kgp] output-projection operand (feature hi/lo halves)
   __half *wT;      // [Cout_pad, Kgp] output-projection weights, K-major
   uint8_t *rowflag;// [B*N] row has a non-empty neighbourhood
-  float *part;     // [gemm_ks, B*N, Cout_pad] split-K partial sums of the projection
 };
 
 struct Outputs {
@@ -92,7 +91,6 @@ cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cuda
 cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                         const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
                         const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s);
-cudaError_t launch_weight_prep(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s);
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl,
                             cudaStream_t s);

@@ -133,7 +133,6 @@ FIPA_API fipa_status fipa_forward_noalloc(fipa_dtype dtype, const void* q, const
   w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
   w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
   w.rowflag = ws + p.off_rowflag;
-  w.part = reinterpret_cast<float*>(ws + p.off_part);
 
   fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
                   w_out, b_out, (float)eps};
@@ -153,7 +152,6 @@ FIPA_API fipa_status fipa_forward_noalloc(fipa_dtype dtype, const void* q, const
   if (cudaMemsetAsync(ds->status, 0, sizeof(int), s) != cudaSuccess) return FIPA_ERR_CUDA;
   if (fipa::launch_prologue(p, in, w, s) != cudaSuccess) return FIPA_ERR_CUDA;
   if (fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s) != cudaSuccess) return FIPA_ERR_CUDA;
-  if (fipa::launch_weight_prep(p, in, w, s) != cudaSuccess) return FIPA_ERR_CUDA;
   if (fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s) != cudaSuccess) return FIPA_ERR_CUDA;
   return FIPA_OK;
 }

@@ -106,10 +106,12 @@ struct Plan {
   int gemm_nks;       // K chunks per split
   int gemm_nst;
   size_t gemm_smem;
+  int wp_ctas;        // weight-preparation CTAs at the front of the prologue launch
+  int lift_ctas;      // lift CTAs per sample (kLiftRes residues each)
   // workspace byte offsets
   size_t off_Q, off_KH, off_VH, off_Z, off_kvec, off_qvec, off_orig, off_flag;
   size_t off_QP, off_KP;
-  size_t off_stats, off_feat, off_wT, off_rowflag, off_part, total;
+  size_t off_stats, off_feat, off_wT, off_rowflag, total;
 };
 
 // Returns 0 and fills `p`, or a nonzero reason code: 1 = bad dims, 2 = unsupported.
@@ -193,15 +195,19 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.Kg = H * p.nseg * p.Wh8;
   p.Kgp = rup(p.Kg, kChunk);
   // N tile and split-K so that the grid covers the SMs (deterministic split-K:
-  // partial sums go to the workspace and a reduce kernel adds them in order)
+  // the splits of an output tile form one thread-block cluster and add their
+  // partial tiles in split order through distributed shared memory)
   {
     // N tile = all of Cout up to 256 (wide MMAs); split-K fills the SMs
     const int mt = cdiv(B * N, kTile), nk = p.Kgp / kChunk;
     const int nt_w = Cout >= 256 ? 256 : rup(Cout, 16);
     p.ntile_out = nt_w;
     const int tiles = mt * cdiv(Cout, nt_w);
+    // split-K factor: fill the SMs, at least 4 K chunks per split, and at most
+    // 8 splits (the splits of a tile form one portable-size cluster)
     int ks = tiles >= 148 ? 1 : cdiv(148, tiles);
     if (ks > nk / 4) ks = nk / 4 > 1 ? nk / 4 : 1;
+    if (ks > 8) ks = 8;
     p.gemm_nks = cdiv(nk, ks);
     p.gemm_ks = cdiv(nk, p.gemm_nks);
     size_t stage = 16384 + (size_t)p.ntile_out * 128;
@@ -209,6 +215,9 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
     p.gemm_nst = g > 8 ? 8 : g;
     p.gemm_smem = 2048 + stage * p.gemm_nst;
   }
+  p.wp_ctas = cdiv(p.F, 32) * cdiv(rup(Cout, p.ntile_out), 32);
+  p.lift_ctas = cdiv(N, kLiftRes);
+  if (p.lift_smem < 32 * 33 * 4) p.lift_smem = 32 * 33 * 4;   // the weight-prep tile
   // workspace layout
   const size_t BN = (size_t)B * N, BHN = (size_t)B * H * N;
   size_t o = 0;
@@ -227,7 +236,6 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.off_feat = take(BN * p.Kgp * 2);
   p.off_wT = take((size_t)rup(Cout, p.ntile_out) * p.Kgp * 2);
   p.off_rowflag = take(BN);
-  p.off_part = take(p.gemm_ks > 1 ? (size_t)p.gemm_ks * BN * rup(Cout, p.ntile_out) * 4 : 0);
   p.total = o;
   return 0;
 }

@@ -1,20 +1,19 @@
 // prologue.cu -- frames to global points and the lifted Q / K / V rows (HBM-bound).
 //
-// Two kernels:
-//   origin: one CTA per (128-residue tile, sample) reduces the origin o_G of
-//           each 32-residue group (mean translation of its valid residues) and
-//           the tile's valid flag;
-//   lift:   one CTA per 8 residues of a sample, all heads.  It stages the
-//           frames, z1 rows and Wb^T in shared memory, applies every frame
-//           T_i(x) = R_i x + t_i (page "Invariant point attention (IPA)",
-//           Required behavior: column-vector convention) to all query / key /
-//           value points in parallel, and then writes every lifted row of
-//           plan.h as 16-byte chunks of 8 fp16 values.  Each column segment is
-//           padded to a multiple of 8, so a chunk never straddles two segments.
+// One launch: CTAs that prepare the output weights (wprep.cuh), then one lift
+// CTA per 8 residues of a sample, all heads.  A lift CTA reduces the origin o_G
+// of its 32-residue group (mean translation of its valid residues) and the
+// valid flag of its 128-residue tile; it stages the frames, z1 rows and Wb^T in
+// shared memory, applies every frame T_i(x) = R_i x + t_i (page "Invariant
+// point attention (IPA)", Required behavior: column-vector convention) to all
+// query / key / value points in parallel, and then writes every lifted row of
+// plan.h as 16-byte chunks of 8 fp16 values.  Each column segment is padded to
+// a multiple of 8, so a chunk never straddles two segments.
 // The distance weight g is folded into the query point columns, following the
 // squared-norm expansion of FlashIPA's lifted attention.
 #include "kernels.h"
 #include "sm100.cuh"
+#include "wprep.cuh"
 
 namespace fipa {
 namespace {
@@ -43,35 +42,6 @@ struct PrologueArgs {
   Inputs in;
   Work w;
 };
-
-template <typename T>
-__global__ void __launch_bounds__(kTile) fipa_origin_kernel(const PrologueArgs a) {
-  // warp w reduces 32-residue group 4t+w of the 128-residue tile t
-  const Plan& p = a.p;
-  const T* tr = static_cast<const T*>(a.in.trans);
-  const int t = blockIdx.x, b = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __shared__ int s_any[kTile / 32];
-  float sx = 0.f, sy = 0.f, sz = 0.f, cnt = 0.f;
-  const int i = t * kTile + threadIdx.x;
-  if (i < p.N && a.in.mask[(size_t)b * p.N + i]) {
-    const size_t o = ((size_t)b * p.N + i) * 3;
-    sx = ld_in(tr, o + 0); sy = ld_in(tr, o + 1); sz = ld_in(tr, o + 2); cnt = 1.f;
-  }
-  for (int off = 16; off; off >>= 1) {
-    sx += __shfl_xor_sync(0xffffffffu, sx, off);
-    sy += __shfl_xor_sync(0xffffffffu, sy, off);
-    sz += __shfl_xor_sync(0xffffffffu, sz, off);
-    cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
-  }
-  if (lane == 0) {
-    const float inv = cnt > 0.f ? 1.f / cnt : 0.f;
-    a.w.orig[(size_t)b * p.nG + t * 4 + warp] = make_float4(sx * inv, sy * inv, sz * inv, cnt);
-    s_any[warp] = cnt > 0.f;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) a.w.flag[(size_t)b * p.nT + t] = (s_any[0] | s_any[1] | s_any[2] | s_any[3]) ? 1 : 0;
-}
-
 
 // ---- lift: chunk descriptors
 // Every 16-byte chunk (8 fp16 columns) of a lifted row reads 8 consecutive
@@ -244,13 +214,22 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   const T* Wb = static_cast<const T*>(a.in.Wb);
   const T* raw = static_cast<const T*>(a.in.raw);
   const int N = p.N, H = p.H, P = p.P, Q = p.Q, Cz = p.Cz, RCz = p.R * p.Cz;
-  const int b = blockIdx.y, i0 = blockIdx.x * kLiftRes;
+  extern __shared__ float4 sh4[];
+  if ((int)blockIdx.x < p.wp_ctas) {
+    // output-weight preparation (independent of the lift)
+    const int nbx = cdiv(p.F, 32), cout_pad = rup(p.Cout, p.ntile_out);
+    const int by = blockIdx.x / nbx, bx = blockIdx.x - by * nbx;
+    weight_prep_tile(p, static_cast<const T*>(a.in.w_out), a.w.wT, cout_pad, bx, by,
+                     reinterpret_cast<float (*)[33]>(sh4));
+    return;
+  }
+  const int lid = blockIdx.x - p.wp_ctas;
+  const int b = lid / p.lift_ctas, i0 = (lid - b * p.lift_ctas) * kLiftRes;
   const int nres = min(kLiftRes, N - i0);
   const int RH = nres * H;
   const int PW = 2 * p.P38 + p.Q38;            // point row: [a' | b' | g'], each segment zero-padded
   const int nQ8 = p.Kq >> 3, nK8 = p.KHp >> 3, nV8 = p.VHp >> 3, nZ8 = p.Zp >> 3;
 
-  extern __shared__ float4 sh4[];
   float* wbt = reinterpret_cast<float*>(sh4);                // [H][Cz]  Wb^T / sqrt(3)
   float* z1s = wbt + rup(H * Cz, 8);                         // [8][RC8]
   float* z2s = z1s + kLiftRes * p.RC8;                       // [8][RC8]
@@ -262,6 +241,44 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   uint32_t* tab = reinterpret_cast<uint32_t*>(frm + kLiftRes * 12);   // chunk descriptors Q | K | V | Z
   __shared__ float s_gamma[64];
   __shared__ int s_valid[kLiftRes];
+  __shared__ float4 s_orig;
+
+  // ---- phase 0: origin o_G of this CTA's 32-residue group (mean translation
+  // of its valid residues; its CTA at the group start writes it for the core),
+  // and the valid flag of the 128-residue tile (written by its first CTA)
+  const int warp0 = threadIdx.x >> 5, lane0 = threadIdx.x & 31;
+  if (warp0 == 0) {
+    const int g = i0 / kGroup, i = g * kGroup + lane0;
+    float sx = 0.f, sy = 0.f, sz = 0.f, cnt = 0.f;
+    if (i < N && a.in.mask[(size_t)b * N + i]) {
+      const size_t o = ((size_t)b * N + i) * 3;
+      sx = ld_in(tr, o + 0); sy = ld_in(tr, o + 1); sz = ld_in(tr, o + 2); cnt = 1.f;
+    }
+    for (int off = 16; off; off >>= 1) {
+      sx += __shfl_xor_sync(0xffffffffu, sx, off);
+      sy += __shfl_xor_sync(0xffffffffu, sy, off);
+      sz += __shfl_xor_sync(0xffffffffu, sz, off);
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    }
+    if (lane0 == 0) {
+      const float inv = cnt > 0.f ? 1.f / cnt : 0.f;
+      s_orig = make_float4(sx * inv, sy * inv, sz * inv, cnt);
+      if (i0 % kGroup == 0) a.w.orig[(size_t)b * p.nG + g] = s_orig;
+    }
+  } else if (warp0 == 1 && i0 % kTile == 0) {
+    bool any = false;
+    for (int k = lane0; k < kTile; k += 32) {
+      const int i = i0 + k;
+      any |= i < N && a.in.mask[(size_t)b * N + i] != 0;
+    }
+    any = __any_sync(0xffffffffu, any);
+    if (lane0 == 0) a.w.flag[(size_t)b * p.nT + i0 / kTile] = any ? 1 : 0;
+    // groups of this tile that lie wholly past N have no lift CTA: their
+    // origin is 0 with no valid residue (every tile's four are read by the core)
+    if (lane0 < kTile / kGroup && i0 + lane0 * kGroup >= N)
+      a.w.orig[(size_t)b * p.nG + i0 / kGroup + lane0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  __syncthreads();
 
   // ---- phase 1: stage the inputs of the 8 residues, zero the point rows,
   // build the chunk table (independent work, issued together)
@@ -285,7 +302,7 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     if (c < 9) {
       frm[e] = ld_in(rot, bi * 9 + c);
     } else {
-      const float4 o = a.w.orig[(size_t)b * p.nG + (i0 + r) / kGroup];
+      const float4 o = s_orig;                  // all kLiftRes residues share one group
       frm[e] = ld_in(tr, bi * 3 + (c - 9)) - (c == 9 ? o.x : c == 10 ? o.y : o.z);
     }
   }
@@ -390,21 +407,17 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
 }  // namespace
 
 cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s) {
+  // one launch: the weight-preparation CTAs first, then B x lift_ctas lift CTAs
   PrologueArgs a{p, in, w};
-  dim3 g1(p.nT, p.B), g2((p.N + kLiftRes - 1) / kLiftRes, p.B);
-  if (p.f32) {
-    fipa_origin_kernel<float><<<g1, kTile, 0, s>>>(a);
-    auto kfn = fipa_lift_kernel<float>;
-    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
-    if (e != cudaSuccess) return e;
-    kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
-  } else {
-    fipa_origin_kernel<__nv_bfloat16><<<g1, kTile, 0, s>>>(a);
-    auto kfn = fipa_lift_kernel<__nv_bfloat16>;
-    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
-    if (e != cudaSuccess) return e;
-    kfn<<<g2, kLiftThreads, p.lift_smem, s>>>(a);
-  }
+  const unsigned grid = (unsigned)(p.wp_ctas + (size_t)p.B * p.lift_ctas);
+  const void* kfn = p.f32 ? reinterpret_cast<const void*>(fipa_lift_kernel<float>)
+                          : reinterpret_cast<const void*>(fipa_lift_kernel<__nv_bfloat16>);
+  cudaError_t e = allow_max_smem(kfn);
+  if (e != cudaSuccess) return e;
+  if (p.f32)
+    fipa_lift_kernel<float><<<grid, kLiftThreads, p.lift_smem, s>>>(a);
+  else
+    fipa_lift_kernel<__nv_bfloat16><<<grid, kLiftThreads, p.lift_smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -193,15 +193,15 @@ class Fipa:
         self._check(st)
         return out
 
-    STAGES = ("prologue", "core", "weight_prep", "out_proj", "attention")
+    STAGES = ("prologue", "core", "out_proj", "attention")
 
     def enable_stage_timing(self, enable: bool = True):
         self._check(self.lib.fipa_enable_stage_timing(self.handle, 1 if enable else 0))
 
     def stage_times(self) -> dict:
         """Device ms of each stage of the most recent timed forward."""
-        buf = (ctypes.c_float * 5)()
-        self._check(self.lib.fipa_stage_times(self.handle, buf, 5))
+        buf = (ctypes.c_float * len(self.STAGES))()
+        self._check(self.lib.fipa_stage_times(self.handle, buf, len(self.STAGES)))
         return dict(zip(self.STAGES, [float(x) for x in buf]))
 
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
