@@ -728,49 +728,60 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   ttr.ev(42);
   const EpiLayout el = epi_layout(p, a.z1);
   const bool fast_pair = el.fast_pair;
-  if (warp >= 4 && *abort_flag == 0) {
-    const int wq = warp - 4;
+  // per-row state for the warps that did not run the softmax (the key-term
+  // buffer is free now); the z1 copies of the softmax threads complete first
+  float2* rowinfo = reinterpret_cast<float2*>(tail + kKtBuf);
+  if (warp >= 4) {
+    cp_async_wait_all();
+    rowinfo[(warp - 4) * 32 + lane] = make_float2(rowL, (row_ok && nkt > 0) ? 1.f : 0.f);
+  }
+  __syncthreads();
+  if (*abort_flag == 0) {
+    // warps w and w+4 serve the same 32 rows (TMEM lane quadrant w % 4):
+    // warps 4-7 the scalar, point and length features, warps 0-3 the pair block
+    const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int i = qt * kTile + r;
     const bool in_range = i < N;
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
-    const int staged = el.staged;                           // columns staged in shared memory
-    float* orow = reinterpret_cast<float*>(smem + el.o_off) + (size_t)r * (staged + 1);
-    const float inv = rowL > 0.f ? 1.f / rowL : 0.f;
-    const bool live = row_ok && nkt > 0;
-    if (live) {
-      for (int c = 0; c < staged; c += 32) {
-        uint32_t o[32];
-        tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv;
-      }
-    }
-    ttr.ev(45);
+    const float2 ri = rowinfo[r];
+    const float inv = ri.x > 0.f ? 1.f / ri.x : 0.f;
+    const bool live = ri.y != 0.f;
+    const bool empty = !(ri.x > 0.f) || !live;
     const size_t bi = (size_t)b * N + (in_range ? i : 0);
-    const bool empty = !(rowL > 0.f) || !live;
     // this row's head block of the projection operand and its local points
     __half* fblk = a.feat + bi * p.Kgp + (size_t)h * p.nseg * p.Wh8;
-    float* lp = a.local_points + (bi * p.H + h) * (size_t)p.Q * 3;
-    if (in_range) {
-      a.stats[(size_t)bh * N + i] = make_float2(rowM, rowL);
-      if (a.lse != nullptr) {
-        const float4 qv = a.qvec[(size_t)bh * N + i];
-        a.lse[(size_t)bh * N + i] = rowL > 0.f ? (rowM + log2f(rowL)) * kLn2 + qv.w : -INFINITY;
+    if (warp >= 4) {
+      const int staged = el.staged;                         // columns staged in shared memory
+      float* orow = reinterpret_cast<float*>(smem + el.o_off) + (size_t)r * (staged + 1);
+      if (live) {
+        for (int c = 0; c < staged; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv;
+        }
       }
-      if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
-      if (h == 0)
-        for (int c = p.Kg; c < p.Kgp; ++c) a.feat[bi * p.Kgp + c] = __float2half_rn(0.f);
-      write_features(a, bi, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT,
-                     fblk, lp);
-    }
-    ttr.ev(46);
-    if (fast_pair) {
+      ttr.ev(45);
+      float* lp = a.local_points + (bi * p.H + h) * (size_t)p.Q * 3;
+      if (in_range) {
+        a.stats[(size_t)bh * N + i] = make_float2(rowM, rowL);
+        if (a.lse != nullptr) {
+          const float4 qv = a.qvec[(size_t)bh * N + i];
+          a.lse[(size_t)bh * N + i] = rowL > 0.f ? (rowM + log2f(rowL)) * kLn2 + qv.w : -INFINITY;
+        }
+        if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
+        if (h == 0)
+          for (int c = p.Kg; c < p.Kgp; ++c) a.feat[bi * p.Kgp + c] = __float2half_rn(0.f);
+        write_features(a, bi, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT,
+                       fblk, lp);
+      }
+      ttr.ev(46);
+    } else if (fast_pair) {
       // pair block straight from tensor memory, 32 channels at a time
       const int Cz = p.Cz, RCz = p.R * Cz, pcol = p.Dv + 4 * p.Q;
       __half* frow = fblk;
-      cp_async_wait_all();
       const uint8_t* zs = smem + (size_t)r * el.z1_stride;
       for (int c0 = 0; c0 < Cz; c0 += 32) {
         float acc[32];
@@ -822,8 +833,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (in_range) put_run32(frow, p.Wh8, p.f32, pcol + c0, acc);
       }
     }
-    ttr.ev(47);
   }
+  ttr.ev(47);
   // ---------------------------------------------------------------- teardown
   ttr.ev(43);
   tc_fence_before();
