@@ -170,6 +170,14 @@ fipa_status fipa_forward_noalloc(fipa_dtype dtype,
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */
 fipa_status fipa_sync_status(fipa_handle* h, void* stream);
 
+/* Failure-path self-test.  Launches on `stream` one CTA whose bounded wait on
+ * an mbarrier that nothing completes runs out after `timeout_ms` (1..10000):
+ * the kernel records FIPA_ERR_DEVICE_TIMEOUT in the handle's status word and
+ * returns, exactly as a real wait of any library kernel would, without a
+ * fault or a hang; the next fipa_sync_status reports it and clears the word.
+ * Returns FIPA_ERR_INVALID_ARG for a null handle or an out-of-range timeout. */
+fipa_status fipa_selftest_timeout(fipa_handle* h, unsigned timeout_ms, void* stream);
+
 /* Profiling aid (stage timing).  With `enable` nonzero, later fipa_forward
  * calls on this handle record a CUDA event before and after each of their
  * kernels on the call's stream; the events are created here, so fipa_forward

@@ -9,6 +9,7 @@
 
 #include "fipa.h"
 #include "kernels.h"
+#include "sm100.cuh"
 
 #define FIPA_API extern "C" __attribute__((visibility("default")))
 
@@ -251,6 +252,33 @@ FIPA_API fipa_status fipa_sync_status(fipa_handle* h, void* stream) {
     std::snprintf(buf, sizeof(buf), "device wait timed out (code %d, site %d)", code & 0xff, code >> 8);
     return fail(h, FIPA_ERR_DEVICE_TIMEOUT, buf);
   }
+  return FIPA_OK;
+}
+
+namespace {
+// One CTA whose thread 0 waits, with the library's bounded wait, on an
+// mbarrier that nothing ever completes: the wait runs out, raises the CTA's
+// abort flag, writes the timeout code into the status word and returns.
+__global__ void fipa_selftest_wait_kernel(int* status, unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    fipa::mbar_init(&bar, 1);
+    fipa::fence_mbar_init();
+    abort_flag = 0;
+    const fipa::WaitCtx wc{&abort_flag, status, timeout_ns};
+    fipa::mbar_wait(&bar, 0, wc, 63);
+  }
+}
+}  // namespace
+
+FIPA_API fipa_status fipa_selftest_timeout(fipa_handle* h, unsigned timeout_ms, void* stream) {
+  if (h == nullptr || timeout_ms == 0 || timeout_ms > 10000) return FIPA_ERR_INVALID_ARG;
+  DeviceGuard g(h->device);
+  fipa_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      h->d_status, (unsigned long long)timeout_ms * 1000000ull);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(h, "self-test launch", e);
   return FIPA_OK;
 }
 

@@ -60,6 +60,8 @@ def load_library():
     lib.fipa_forward.restype = c_int
     lib.fipa_sync_status.argtypes = [vp, vp]
     lib.fipa_sync_status.restype = c_int
+    lib.fipa_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
+    lib.fipa_selftest_timeout.restype = c_int
     lib.fipa_status_string.argtypes = [c_int]
     lib.fipa_status_string.restype = ctypes.c_char_p
     lib.fipa_last_error.argtypes = [vp]
@@ -207,6 +209,11 @@ class Fipa:
     def sync_status(self, stream: Optional[torch.cuda.Stream] = None):
         s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))
         self._check(self.lib.fipa_sync_status(self.handle, ctypes.c_void_p(s.cuda_stream)))
+
+    def selftest_timeout(self, timeout_ms: int, stream: Optional[torch.cuda.Stream] = None):
+        """Launch the failure-path self-test (a bounded wait that runs out)."""
+        s = stream if stream is not None else torch.cuda.current_stream(torch.device("cuda", self.device))
+        self._check(self.lib.fipa_selftest_timeout(self.handle, int(timeout_ms), ctypes.c_void_p(s.cuda_stream)))
 
 
 NOALLOC_SCRATCH_BYTES = 32 << 20
