@@ -40,6 +40,7 @@ constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
 constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
 constexpr int kLiftRes = 8;      // residues per prologue lift CTA (divides the 128-residue tile)
+constexpr int kWpTiles = 4;      // 32x32 output-weight tiles per weight-preparation CTA
 
 #ifdef __CUDACC__
 #define FIPA_HD __host__ __device__
@@ -178,9 +179,9 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)(p.nQc + nst) * 16384) {
     *why = "value width too large for the epilogue staging"; return 2;
   }
-  // prologue lift kernel: Wb^T, zero-padded z1 / z2 / q / k / v / point rows
+  // prologue lift kernel: Wb^T, zero-padded z1 / q / k / v / point rows
   // and frames of kLiftRes residues, and the chunk table of the four row types
-  p.lift_smem = ((size_t)rup(H * Cz, 8) + (size_t)kLiftRes * 2 * p.RC8 +
+  p.lift_smem = ((size_t)rup(H * Cz, 8) + (size_t)kLiftRes * p.RC8 +
                  (size_t)kLiftRes * H * (2 * p.D8 + p.Dv8 + 2 * p.P38 + p.Q38) + kLiftRes * 12) * 4 +
                 (size_t)(p.Kq + p.KHp + p.VHp + p.Zp) / 8 * 4;
   p.fd_H = make_fastdiv(H); p.fd_P = make_fastdiv(P); p.fd_Q = make_fastdiv(Q); p.fd_Cz = make_fastdiv(Cz);
@@ -215,7 +216,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
     p.gemm_nst = g > 8 ? 8 : g;
     p.gemm_smem = 2048 + stage * p.gemm_nst;
   }
-  p.wp_ctas = cdiv(p.F, 32) * cdiv(rup(Cout, p.ntile_out), 32);
+  p.wp_ctas = cdiv(cdiv(p.F, 32) * cdiv(rup(Cout, p.ntile_out), 32), kWpTiles);
   p.lift_ctas = cdiv(N, kLiftRes);
   if (p.lift_smem < 32 * 33 * 4) p.lift_smem = 32 * 33 * 4;   // the weight-prep tile
   // workspace layout

@@ -173,8 +173,8 @@ __device__ __forceinline__ void stage_rows(float* dst, int L8, const FastDiv& fd
 
 // The 8 fp32 values of one chunk of a lifted row (all zero for a masked residue).
 __device__ __forceinline__ void chunk_values(uint32_t d, bool valid, const float* scal, const float* prow,
-                                             float ptscale, const float* z1row, const float* z2row,
-                                             const float* wrow, int Cz, bool cz8, float (&v)[8]) {
+                                             float ptscale, const float* z1row, const float* wrow, int Cz, bool cz8,
+                                             float (&v)[8]) {
   const uint32_t src = valid ? (d >> 22) & 15u : (uint32_t)kSrcZero;
   const int off = d & 2047, woff = (d >> 11) & 2047;
   if (src == kSrcScalar) {
@@ -195,8 +195,6 @@ __device__ __forceinline__ void chunk_values(uint32_t d, bool valid, const float
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t) v[t] *= w[t];
-  } else if (src == kSrcZ2) {
-    lds8(z2row + off, v);
   } else {
 #pragma unroll
     for (int t = 0; t < 8; ++t) v[t] = 0.f;
@@ -218,9 +216,13 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   if ((int)blockIdx.x < p.wp_ctas) {
     // output-weight preparation (independent of the lift)
     const int nbx = cdiv(p.F, 32), cout_pad = rup(p.Cout, p.ntile_out);
-    const int by = blockIdx.x / nbx, bx = blockIdx.x - by * nbx;
-    weight_prep_tile(p, static_cast<const T*>(a.in.w_out), a.w.wT, cout_pad, bx, by,
-                     reinterpret_cast<float (*)[33]>(sh4));
+    const int ntiles = nbx * cdiv(cout_pad, 32);
+    for (int t = blockIdx.x * kWpTiles; t < min(ntiles, (int)(blockIdx.x + 1) * kWpTiles); ++t) {
+      const int by = t / nbx, bx = t - by * nbx;
+      weight_prep_tile(p, static_cast<const T*>(a.in.w_out), a.w.wT, cout_pad, bx, by,
+                       reinterpret_cast<float (*)[33]>(sh4));
+      __syncthreads();                      // the tile buffer is reused by the next tile
+    }
     return;
   }
   const int lid = blockIdx.x - p.wp_ctas;
@@ -232,8 +234,7 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
 
   float* wbt = reinterpret_cast<float*>(sh4);                // [H][Cz]  Wb^T / sqrt(3)
   float* z1s = wbt + rup(H * Cz, 8);                         // [8][RC8]
-  float* z2s = z1s + kLiftRes * p.RC8;                       // [8][RC8]
-  float* qs = z2s + kLiftRes * p.RC8;                        // [8*H][D8]  q / sqrt(3D)
+  float* qs = z1s + kLiftRes * p.RC8;                        // [8*H][D8]  q / sqrt(3D)
   float* ks = qs + kLiftRes * H * p.D8;                      // [8*H][D8]
   float* vs = ks + kLiftRes * H * p.D8;                      // [8*H][Dv8]
   float* pts = vs + kLiftRes * H * p.Dv8;                    // [8*H][PW]  global point - o_G
@@ -278,10 +279,10 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     if (lane0 < kTile / kGroup && i0 + lane0 * kGroup >= N)
       a.w.orig[(size_t)b * p.nG + i0 / kGroup + lane0] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __syncthreads();
 
-  // ---- phase 1: stage the inputs of the 8 residues, zero the point rows,
-  // build the chunk table (independent work, issued together)
+  // ---- phase 1 (with phase 0 above): stage the inputs of the 8 residues,
+  // zero the point rows, build the chunk table (independent work, issued
+  // together)
   const float inv_sqrt3 = rsqrtf(3.0f);
   const size_t bi0 = (size_t)b * N + i0;
   for (uint32_t e = threadIdx.x; e < (uint32_t)(H * Cz); e += blockDim.x) {
@@ -289,7 +290,6 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     wbt[e] = ld_in(Wb, (size_t)c * H + h) * inv_sqrt3;
   }
   stage_rows(z1s, p.RC8, p.fd_RC8v, static_cast<const T*>(a.in.z1) + bi0 * RCz, RCz, nres, 1.f);
-  stage_rows(z2s, p.RC8, p.fd_RC8v, static_cast<const T*>(a.in.z2) + bi0 * RCz, RCz, nres, 1.f);
   stage_rows(qs, p.D8, p.fd_D8v, static_cast<const T*>(a.in.q) + bi0 * H * p.D, p.D, RH,
              rsqrtf(3.0f * (float)p.D));
   stage_rows(ks, p.D8, p.fd_D8v, static_cast<const T*>(a.in.k) + bi0 * H * p.D, p.D, RH, 1.f);
@@ -299,12 +299,7 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   for (int e = threadIdx.x; e < nres * 12; e += blockDim.x) {
     const int r = e / 12, c = e - r * 12;
     const size_t bi = bi0 + r;
-    if (c < 9) {
-      frm[e] = ld_in(rot, bi * 9 + c);
-    } else {
-      const float4 o = s_orig;                  // all kLiftRes residues share one group
-      frm[e] = ld_in(tr, bi * 3 + (c - 9)) - (c == 9 ? o.x : c == 10 ? o.y : o.z);
-    }
+    frm[e] = c < 9 ? ld_in(rot, bi * 9 + c) : ld_in(tr, bi * 3 + (c - 9));   // t - o_G in phase 2
   }
   for (int c = threadIdx.x; c < nQ8 + nK8 + nV8 + nZ8; c += blockDim.x) {
     int rt = kRowQ, cc = c;
@@ -320,16 +315,18 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   // ---- phase 2: every point of every head, T_i(x) = R_i x + t_i relative to
   // the group origin (page "Invariant point attention (IPA)", Required
   // behavior: column-vector convention)
+  const float4 og = s_orig;                    // all kLiftRes residues share one group
   auto apply = [&](const T* src, int npts, const FastDiv& fd_npts, int seg_off) {
     for (uint32_t e = threadIdx.x; e < (uint32_t)(RH * npts); e += blockDim.x) {
       const uint32_t rh = fd_npts.div(e), pt = e - rh * npts, r = p.fd_H.div(rh);
       const T* x = src + ((bi0 * H + rh) * npts + pt) * 3;
       const float x0 = ld_in(x, 0), x1 = ld_in(x, 1), x2 = ld_in(x, 2);
       const float* F = frm + r * 12;
+      const float t0 = F[9] - og.x, t1 = F[10] - og.y, t2 = F[11] - og.z;
       float* o = pts + (size_t)rh * PW + seg_off + 3 * pt;
-      o[0] = F[0] * x0 + F[1] * x1 + F[2] * x2 + F[9];
-      o[1] = F[3] * x0 + F[4] * x1 + F[5] * x2 + F[10];
-      o[2] = F[6] * x0 + F[7] * x1 + F[8] * x2 + F[11];
+      o[0] = F[0] * x0 + F[1] * x1 + F[2] * x2 + t0;
+      o[1] = F[3] * x0 + F[4] * x1 + F[5] * x2 + t1;
+      o[2] = F[6] * x0 + F[7] * x1 + F[8] * x2 + t2;
     }
   };
   apply(qp, P, p.fd_P, 0);
@@ -376,30 +373,45 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     const uint32_t d = tab[c];
     float v[8];
     chunk_values(d, s_valid[r] != 0, qs + (size_t)rh * p.D8, pts + (size_t)rh * PW, 2.f * s_gamma[h < 64 ? h : 63],
-                 z1s + (size_t)r * p.RC8, nullptr, wbt + (size_t)h * Cz, Cz, cz8, v);
+                 z1s + (size_t)r * p.RC8, wbt + (size_t)h * Cz, Cz, cz8, v);
     stg8_half(a.w.Q + (((size_t)b * H + h) * N + i0 + r) * p.Kq + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
   for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nK8; e += nthr) {
     const uint32_t rh = p.fd_nK8.div(e), c = e - rh * nK8, r = p.fd_H.div(rh), h = rh - r * H;
     const uint32_t d = tab[nQ8 + c];
     float v[8];
-    chunk_values(d, s_valid[r] != 0, ks + (size_t)rh * p.D8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr,
-                 nullptr, Cz, cz8, v);
+    chunk_values(d, s_valid[r] != 0, ks + (size_t)rh * p.D8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr, Cz,
+                 cz8, v);
     stg8_half(a.w.KH + (((size_t)b * H + h) * N + i0 + r) * p.KHp + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
   for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nV8; e += nthr) {
     const uint32_t rh = p.fd_nV8.div(e), c = e - rh * nV8, r = p.fd_H.div(rh), h = rh - r * H;
     const uint32_t d = tab[nQ8 + nK8 + c];
     float v[8];
-    chunk_values(d, s_valid[r] != 0, vs + (size_t)rh * p.Dv8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr,
-                 nullptr, Cz, cz8, v);
+    chunk_values(d, s_valid[r] != 0, vs + (size_t)rh * p.Dv8, pts + (size_t)rh * PW, 1.f, nullptr, nullptr, Cz,
+                 cz8, v);
     stg8_half(a.w.VH + (((size_t)b * H + h) * N + i0 + r) * p.VHp + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
+  // pair-factor rows read z2 straight from global memory (one use per value)
+  const T* z2 = static_cast<const T*>(a.in.z2);
+  const bool z2vec = (RCz & 7) == 0 && (reinterpret_cast<uintptr_t>(z2) & 15) == 0;
   for (uint32_t e = threadIdx.x; e < (uint32_t)nres * nZ8; e += nthr) {
     const uint32_t r = p.fd_nZ8.div(e), c = e - r * nZ8;
     const uint32_t d = tab[nQ8 + nK8 + nV8 + c];
     float v[8];
-    chunk_values(d, s_valid[r] != 0, nullptr, nullptr, 1.f, nullptr, z2s + (size_t)r * p.RC8, nullptr, Cz, cz8, v);
+    const int off = d & 2047;
+    if (s_valid[r] != 0 && ((d >> 22) & 15u) == kSrcZ2) {
+      const T* zr = z2 + (bi0 + r) * RCz + off;
+      if (z2vec && off + 8 <= RCz) {
+        ldg8(zr, v);
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] = off + t < RCz ? ld_in(zr, t) : 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) v[t] = 0.f;
+    }
     stg8_half(a.w.Z + (bi0 + r) * p.Zp + ((size_t)c << 3), v, (d >> 26) & 1u);
   }
 }
