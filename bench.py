@@ -47,7 +47,7 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="0, 1, 2, 4 or 3-<N> (length sweep, N in 512..16384)")
     ap.add_argument("--impl", choices=("fipa", "reference"), default="fipa")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true",
@@ -332,23 +332,71 @@ def run_fipa(args, wl, rank, world, local_rank):
     h.enable_stage_timing(False)
     core_ms = stage_sum["core"] / nb
 
-    # ---- end to end through the public API: pinned host inputs -> device -> result on host
-    host_in = {k: v.cpu().pin_memory() for k, v in d_in.items() if v is not None}
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items()}
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    # ---- end to end through the public API: each step copies its inputs from
+    # pinned host memory (one packed buffer), runs the forward and copies the
+    # update and local points back (one packed buffer).  Two steps are in
+    # flight: step k+1's upload and step k-1's download overlap step k's
+    # forward (separate copy streams, two device buffer sets, event-ordered).
     h.enable_stage_timing(False)
-    e2e_steps = max(1, min(args.e2e_steps, args.steps))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    names = [k for k, v in d_in.items() if v is not None]
+
+    def packed_layout(tensors):
+        offs, o = {}, 0
+        for k, t in tensors.items():
+            offs[k] = o
+            o = (o + t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, o
+
+    in_offs, in_bytes = packed_layout({k: d_in[k] for k in names})
+    out_offs, out_bytes = packed_layout(out)
+    host_in = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+    for k in names:
+        t = d_in[k].cpu().contiguous().view(torch.uint8).reshape(-1)
+        host_in[in_offs[k]:in_offs[k] + t.numel()].copy_(t)
+    host_out = [torch.empty(out_bytes, dtype=torch.uint8).pin_memory() for _ in range(2)]
+
+    def views(buf, offs, like):
+        return {k: buf[offs[k]:offs[k] + like[k].numel() * like[k].element_size()].view(like[k].dtype)
+                .reshape(like[k].shape) for k in offs}
+
+    dbuf_in = [torch.empty(in_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dbuf_out = [torch.empty(out_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dev_in = [dict(views(b, in_offs, {k: d_in[k] for k in names}), pair_mask=None) if "pair_mask" not in names
+              else views(b, in_offs, {k: d_in[k] for k in names}) for b in dbuf_in]
+    dev_out = [views(b, out_offs, out) for b in dbuf_out]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_fwd = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    h2d, d2h = in_bytes, out_bytes
+    e2e_steps = max(2, min(args.e2e_steps, args.steps))
+
+    def e2e_step(k):
+        j = k % 2
+        if k >= 2:
+            s_in.wait_event(ev_fwd[j])          # forward k-2 has read buffer j
+        with torch.cuda.stream(s_in):
+            dbuf_in[j].copy_(host_in, non_blocking=True)
+            ev_in[j].record(s_in)
+        stream.wait_event(ev_in[j])
+        if k >= 2:
+            stream.wait_event(ev_out[j])        # download k-2 has read output j
+        h.forward(dev_in[j], eps=inp["eps"], workspace=workspace, out=dev_out[j], stream=stream)
+        ev_fwd[j].record(stream)
+        s_out.wait_event(ev_fwd[j])
+        with torch.cuda.stream(s_out):
+            host_out[j].copy_(dbuf_out[j], non_blocking=True)
+            ev_out[j].record(s_out)
+
+    for k in range(2):                          # warm-up (first-call host setup)
+        e2e_step(k)
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        for k, v in host_in.items():
-            d_in[k].copy_(v, non_blocking=True)
-        forward()
-        for k, v in host_out.items():
-            v.copy_(out[k], non_blocking=True)
-    e1.record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    s_out.wait_stream(stream)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, dev)
@@ -426,7 +474,9 @@ def main_fipa(args, wl):
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": {"value": padded * world / (r["e2e_ms"] / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "how": "public binding, pinned packed host buffers, one upload and one download per step, "
+                       "two steps in flight (copies overlap the neighbouring forwards)"},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
