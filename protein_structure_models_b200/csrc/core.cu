@@ -169,32 +169,48 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
   }
   // scalar block
   put_run(fblk, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
-  // points: aggregate (hi + lo halves + group-origin part), back into the query
-  // frame; the local coordinates overwrite the consumed hi slots, the lengths the lo slots
+  // points, 8 at a time in registers: aggregate (hi + lo halves + group-origin
+  // part), back into the query frame, lengths; then the x, y, z and length
+  // feature runs and the local points straight from registers
   const int gofs = p.nsv * p.Dv8;
-  for (int q = 0; q < Q; ++q) {
-    const float gx = orow[gofs + 3 * q + 0] + orow[gofs + p.Q38 + 3 * q + 0] + Gx - t[0];
-    const float gy = orow[gofs + 3 * q + 1] + orow[gofs + p.Q38 + 3 * q + 1] + Gy - t[1];
-    const float gz = orow[gofs + 3 * q + 2] + orow[gofs + p.Q38 + 3 * q + 2] + Gz - t[2];
-    const float lx = R[0] * gx + R[3] * gy + R[6] * gz;
-    const float ly = R[1] * gx + R[4] * gy + R[7] * gz;
-    const float lz = R[2] * gx + R[5] * gy + R[8] * gz;
-    orow[gofs + 3 * q + 0] = lx;
-    orow[gofs + 3 * q + 1] = ly;
-    orow[gofs + 3 * q + 2] = lz;
-    orow[gofs + p.Q38 + q] = sqrtf(lx * lx + ly * ly + lz * lz + a.eps);
+  const bool lp_vec = (reinterpret_cast<uintptr_t>(lp) & 15) == 0;
+  for (int q0 = 0; q0 < Q; q0 += 8) {
+    const int nq = min(8, Q - q0);
+    float lx[8], ly[8], lz[8], ln[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      lx[u] = ly[u] = lz[u] = ln[u] = 0.f;
+      if (u < nq) {
+        const int q = q0 + u;
+        const float gx = orow[gofs + 3 * q + 0] + orow[gofs + p.Q38 + 3 * q + 0] + Gx - t[0];
+        const float gy = orow[gofs + 3 * q + 1] + orow[gofs + p.Q38 + 3 * q + 1] + Gy - t[1];
+        const float gz = orow[gofs + 3 * q + 2] + orow[gofs + p.Q38 + 3 * q + 2] + Gz - t[2];
+        lx[u] = R[0] * gx + R[3] * gy + R[6] * gz;
+        ly[u] = R[1] * gx + R[4] * gy + R[7] * gz;
+        lz[u] = R[2] * gx + R[5] * gy + R[8] * gz;
+        ln[u] = sqrtf(lx[u] * lx[u] + ly[u] * ly[u] + lz[u] * lz[u] + a.eps);
+      }
+    }
+    put8(fblk, F, p.f32, xc + q0, nq, lx);
+    put8(fblk, F, p.f32, xc + Q + q0, nq, ly);
+    put8(fblk, F, p.f32, xc + 2 * Q + q0, nq, lz);
+    put8(fblk, F, p.f32, xc + 3 * Q + q0, nq, ln);
+    // local points [q][3] of this chunk: 24 floats, 16-byte stores where aligned
+    float* lq = lp + 3 * q0;
+    if (nq == 8 && lp_vec) {
+      float4* l4 = reinterpret_cast<float4*>(lq);
+      l4[0] = make_float4(lx[0], ly[0], lz[0], lx[1]);
+      l4[1] = make_float4(ly[1], lz[1], lx[2], ly[2]);
+      l4[2] = make_float4(lz[2], lx[3], ly[3], lz[3]);
+      l4[3] = make_float4(lx[4], ly[4], lz[4], lx[5]);
+      l4[4] = make_float4(ly[5], lz[5], lx[6], ly[6]);
+      l4[5] = make_float4(lz[6], lx[7], ly[7], lz[7]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (u < nq) { lq[3 * u] = lx[u]; lq[3 * u + 1] = ly[u]; lq[3 * u + 2] = lz[u]; }
+    }
   }
-  // local points [Q][3]: 16-byte stores where the row allows
-  if (((3 * Q) & 3) == 0 && (reinterpret_cast<uintptr_t>(lp) & 15) == 0) {
-    for (int e = 0; e < 3 * Q; e += 4)
-      *reinterpret_cast<float4*>(lp + e) =
-          make_float4(orow[gofs + e], orow[gofs + e + 1], orow[gofs + e + 2], orow[gofs + e + 3]);
-  } else {
-    for (int e = 0; e < 3 * Q; ++e) lp[e] = orow[gofs + e];
-  }
-  for (int x = 0; x < 3; ++x)
-    put_run(fblk, F, p.f32, xc + x * Q, Q, [&](int q) { return orow[gofs + 3 * q + x]; });
-  put_run(fblk, F, p.f32, xc + 3 * Q, Q, [&](int q) { return orow[gofs + p.Q38 + q]; });
   // pair block through the factors (the tensor-memory path writes it otherwise)
   if (!with_pair) return;
   const int RCz = p.R * Cz;
