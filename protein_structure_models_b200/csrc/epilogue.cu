@@ -216,6 +216,150 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   }
 }
 
+// Persistent form for many output tiles (no split-K, Cout <= one N tile):
+// one CTA per SM loops over tiles t = blockIdx.x, blockIdx.x + gridDim.x, ...
+// TMEM holds two accumulators, so warp 1 runs tile j+1's MMAs while warps
+// 4-7 read tile j's accumulator back, add b_out (staged in shared memory
+// once), zero empty rows and store whole rows as float4 from registers.
+__global__ void __launch_bounds__(256, 1)
+fipa_out_proj_persistent_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                                const ProjArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const Plan& p = a.p;
+  const int nst = p.gemm_nst, ntile = p.ntile_out;
+  const int stage = kChunkBytes + ntile * 128;
+  uint8_t* tail = smem + (size_t)nst * stage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(tail);
+  uint64_t* empty = full + 8;
+  uint64_t* acc_full = full + 16;     // [2]
+  uint64_t* acc_empty = full + 18;    // [2]
+  uint64_t* drain = full + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 256);
+  int* abort_flag = reinterpret_cast<int*>(tail + 260);
+  float* sbias = reinterpret_cast<float*>(tail + 512);   // [ntile]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int M = p.B * p.N, tiles = (M + kTile - 1) / kTile, nk = p.Kgp / kChunk;
+  const uint32_t ncols = ntile <= 32 ? 32 : ntile <= 64 ? 64 : ntile <= 128 ? 128 : 256;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < nst; ++st) { mbar_init(&full[st], 1); mbar_init(&empty[st], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    *abort_flag = 0;
+  }
+  for (int n = threadIdx.x; n < ntile; n += blockDim.x)
+    sbias[n] = n < p.Cout ? (p.f32 ? static_cast<const float*>(a.b_out)[n]
+                                   : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n]))
+                          : 0.f;
+  if (warp == 1) { tmem_alloc(tmem_slot, 2 * ncols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtx wc{abort_flag, a.status, a.timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      int st = 0;
+      uint32_t ph = 0, issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        for (int c = 0; c < nk; ++c) {
+          if (!mbar_wait(&empty[st], ph ^ 1u, wc, 41)) { ok = false; break; }
+          uint8_t* sa = smem + (size_t)st * stage;
+          mbar_arrive_expect_tx(&full[st], (uint32_t)stage);
+          tma_load_2d(sa, &tmA, &full[st], c * kChunk, t * kTile);
+          tma_load_2d(sa + kChunkBytes, &tmB, &full[st], c * kChunk, 0);
+          ++issued;
+          if (++st == nst) { st = 0; ph ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // wait (bounded) for the loads already in flight before the CTA exits
+        const uint32_t last = issued < (uint32_t)nst ? issued : (uint32_t)nst;
+        for (uint32_t k = 0; k < last; ++k) {
+          const uint32_t n = issued - 1 - k;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[n % nst], (n / nst) & 1u) && global_timer_ns() - t0 < a.timeout_ns) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(128, ntile, 0, 0);
+      int st = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int t = blockIdx.x, j = 0; ok && t < tiles; t += gridDim.x, ++j) {
+        const int buf = j & 1;
+        if (!mbar_wait(&acc_empty[buf], ((j >> 1) & 1) ^ 1u, wc, 42)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(buf * ncols);
+        for (int c = 0; c < nk; ++c) {
+          if (!mbar_wait(&full[st], ph, wc, 43)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + (size_t)st * stage);
+          const uint32_t b0 = a0 + kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(acc, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idesc,
+                   (c | kk) != 0 ? 1u : 0u);
+          tc_commit(&empty[st]);
+          if (++st == nst) { st = 0; ph ^= 1u; }
+        }
+        if (ok) tc_commit(&acc_full[buf]);
+      }
+      tc_commit(drain);    // fires once every MMA this thread issued is done
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < a.timeout_ns) {}
+    }
+  } else if (warp >= 4) {
+    const int wq = warp - 4;
+    const bool vec_out = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(a.update) & 15) == 0;
+    for (int t = blockIdx.x, j = 0; t < tiles; t += gridDim.x, ++j) {
+      const int buf = j & 1;
+      bool ok = mbar_wait(&acc_full[buf], (j >> 1) & 1, wc, 44);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int m = t * kTile + wq * 32 + lane;
+      const bool live = m < M;
+      const bool keep = live && a.rowflag[m] != 0;
+      float* urow = a.update + (size_t)(live ? m : 0) * p.Cout;
+      const uint32_t trow = tmem + (uint32_t)(buf * ncols) + ((uint32_t)(wq * 32) << 16);
+      for (int c = 0; c < ntile; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(trow + (uint32_t)c, o);
+        tmem_ld_wait();
+        if (!live) continue;
+        float w[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = keep ? __uint_as_float(o[e]) + sbias[c + e] : 0.f;
+        if (vec_out && c + 32 <= p.Cout) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(urow + c + e) = make_float4(w[e], w[e + 1], w[e + 2], w[e + 3]);
+        } else {
+          for (int e = 0; e < 32; ++e)
+            if (c + e < p.Cout) urow[c + e] = w[e];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * ncols);
+  }
+}
+
 }  // namespace
 
 // Largest split-K factor <= p.gemm_ks whose clusters (one per output tile, of
@@ -265,6 +409,21 @@ cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, cons
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_out_proj_kernel));
   if (e != cudaSuccess) return e;
   const int nk = p.Kgp / kChunk;
+  if (p.gemm_ks == 1 && nt == 1) {
+    static int sm_count[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && sm_count[dev] == 0) cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+    const int sms = (dev >= 0 && dev < 64 && sm_count[dev] > 0) ? sm_count[dev] : 148;
+    if ((int)mt > sms) {
+      const size_t smem = p.gemm_smem + 1024;           // + the staged bias
+      e = cudaFuncSetAttribute(reinterpret_cast<const void*>(fipa_out_proj_persistent_kernel),
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      fipa_out_proj_persistent_kernel<<<(unsigned)sms, 256, smem, s>>>(tmA, tmB, a);
+      return cudaGetLastError();
+    }
+  }
   const int ks = p.gemm_ks > 1 ? resident_split(p, (int)(mt * nt)) : 1;
   a.p.gemm_nks = cdiv(nk, ks);
   a.p.gemm_ks = cdiv(nk, a.p.gemm_nks);
