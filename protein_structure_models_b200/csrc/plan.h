@@ -94,6 +94,7 @@ struct Plan {
   size_t lift_smem;   // dynamic shared memory of the prologue lift kernel
   FastDiv fd_H, fd_P, fd_Q, fd_Cz;               // divisors of the lift kernel's index maps
   FastDiv fd_nQ8, fd_nK8, fd_nV8, fd_nZ8;        // 16-byte chunks per lifted row type
+  FastDiv fd_nQ8e;    // Qhat chunks the lift iterates per row (a u-hi chunk also writes its lo partner)
   FastDiv fd_D8v, fd_Dv8v, fd_RC8v;              // 8-value vectors per staged row
   // Output-projection operand: one block per head, in head order, each block
   // nseg segments (bf16: [hi | lo], f32: [hi | hi | lo]) of Wh8 columns holding
@@ -186,6 +187,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
                 (size_t)(p.Kq + p.KHp + p.VHp + p.Zp) / 8 * 4;
   p.fd_H = make_fastdiv(H); p.fd_P = make_fastdiv(P); p.fd_Q = make_fastdiv(Q); p.fd_Cz = make_fastdiv(Cz);
   p.fd_nQ8 = make_fastdiv(p.Kq / 8); p.fd_nK8 = make_fastdiv(p.KHp / 8);
+  p.fd_nQ8e = make_fastdiv(p.nqz == 2 ? (p.KHp + p.Zp) / 8 : p.Kq / 8);
   p.fd_nV8 = make_fastdiv(p.VHp / 8); p.fd_nZ8 = make_fastdiv(p.Zp / 8);
   p.fd_D8v = make_fastdiv(p.D8 / 8); p.fd_Dv8v = make_fastdiv(p.Dv8 / 8); p.fd_RC8v = make_fastdiv(p.RC8 / 8);
   if (p.lift_smem > 160 * 1024) { *why = "prologue staging exceeds shared memory (H*Cz or R*Cz too large)"; return 2; }

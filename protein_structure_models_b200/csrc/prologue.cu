@@ -368,13 +368,19 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   // chunks of a row
   const bool cz8 = (Cz & 7) == 0;
   const uint32_t nthr = blockDim.x;
-  for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nQ8; e += nthr) {
-    const uint32_t rh = p.fd_nQ8.div(e), c = e - rh * nQ8, r = p.fd_H.div(rh), h = rh - r * H;
+  // with the [u hi | u lo] pair layout a u-hi chunk also writes its lo
+  // partner (the same products, the rounding residual instead of the value)
+  const uint32_t nQ8e = p.fd_nQ8e.d, uhi0 = (uint32_t)p.KHp >> 3, zch = (uint32_t)p.Zp >> 3;
+  const bool pair_lo = p.nqz == 2;
+  for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nQ8e; e += nthr) {
+    const uint32_t rh = p.fd_nQ8e.div(e), c = e - rh * nQ8e, r = p.fd_H.div(rh), h = rh - r * H;
     const uint32_t d = tab[c];
     float v[8];
     chunk_values(d, s_valid[r] != 0, qs + (size_t)rh * p.D8, pts + (size_t)rh * PW, 2.f * s_gamma[h < 64 ? h : 63],
                  z1s + (size_t)r * p.RC8, wbt + (size_t)h * Cz, Cz, cz8, v);
-    stg8_half(a.w.Q + (((size_t)b * H + h) * N + i0 + r) * p.Kq + ((size_t)c << 3), v, (d >> 26) & 1u);
+    __half* qrow = a.w.Q + (((size_t)b * H + h) * N + i0 + r) * p.Kq;
+    stg8_half(qrow + ((size_t)c << 3), v, (d >> 26) & 1u);
+    if (pair_lo && c >= uhi0) stg8_half(qrow + ((size_t)(c + zch) << 3), v, true);
   }
   for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nK8; e += nthr) {
     const uint32_t rh = p.fd_nK8.div(e), c = e - rh * nK8, r = p.fd_H.div(rh), h = rh - r * H;
