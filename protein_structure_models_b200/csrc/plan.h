@@ -39,7 +39,7 @@ constexpr int kMaxPts = 64;      // points per head handled by the prologue scra
 constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
 constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
-constexpr int kLiftRes = 8;      // residues per prologue lift CTA (divides the 128-residue tile)
+constexpr int kLiftRes = 8;      // most residues per prologue lift CTA (divides the 32-residue group)
 constexpr int kWpTiles = 4;      // 32x32 output-weight tiles per weight-preparation CTA
 
 #ifdef __CUDACC__
@@ -109,7 +109,8 @@ struct Plan {
   int gemm_nst;
   size_t gemm_smem;
   int wp_ctas;        // weight-preparation CTAs at the front of the prologue launch
-  int lift_ctas;      // lift CTAs per sample (kLiftRes residues each)
+  int lift_res;       // residues per lift CTA: 4 when that grid still fits about one resident wave, else 8
+  int lift_ctas;      // lift CTAs per sample (lift_res residues each)
   // workspace byte offsets
   size_t off_Q, off_KH, off_VH, off_Z, off_kvec, off_qvec, off_orig, off_flag;
   size_t off_QP, off_KP;
@@ -181,9 +182,10 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
     *why = "value width too large for the epilogue staging"; return 2;
   }
   // prologue lift kernel: Wb^T, zero-padded z1 / q / k / v / point rows
-  // and frames of kLiftRes residues, and the chunk table of the four row types
-  p.lift_smem = ((size_t)rup(H * Cz, 8) + (size_t)kLiftRes * p.RC8 +
-                 (size_t)kLiftRes * H * (2 * p.D8 + p.Dv8 + 2 * p.P38 + p.Q38) + kLiftRes * 12) * 4 +
+  // and frames of lift_res residues, and the chunk table of the four row types
+  p.lift_res = (size_t)B * cdiv(N, 4) <= 148 * 6 ? 4 : kLiftRes;
+  p.lift_smem = ((size_t)rup(H * Cz, 8) + (size_t)p.lift_res * p.RC8 +
+                 (size_t)p.lift_res * H * (2 * p.D8 + p.Dv8 + 2 * p.P38 + p.Q38) + p.lift_res * 12) * 4 +
                 (size_t)(p.Kq + p.KHp + p.VHp + p.Zp) / 8 * 4;
   p.fd_H = make_fastdiv(H); p.fd_P = make_fastdiv(P); p.fd_Q = make_fastdiv(Q); p.fd_Cz = make_fastdiv(Cz);
   p.fd_nQ8 = make_fastdiv(p.Kq / 8); p.fd_nK8 = make_fastdiv(p.KHp / 8);
@@ -219,7 +221,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
     p.gemm_smem = 2048 + stage * p.gemm_nst;
   }
   p.wp_ctas = cdiv(cdiv(p.F, 32) * cdiv(rup(Cout, p.ntile_out), 32), kWpTiles);
-  p.lift_ctas = cdiv(N, kLiftRes);
+  p.lift_ctas = cdiv(N, p.lift_res);
   if (p.lift_smem < 32 * 33 * 4) p.lift_smem = 32 * 33 * 4;   // the weight-prep tile
   // workspace layout
   const size_t BN = (size_t)B * N, BHN = (size_t)B * H * N;

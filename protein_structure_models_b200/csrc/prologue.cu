@@ -226,20 +226,21 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
     return;
   }
   const int lid = blockIdx.x - p.wp_ctas;
-  const int b = lid / p.lift_ctas, i0 = (lid - b * p.lift_ctas) * kLiftRes;
-  const int nres = min(kLiftRes, N - i0);
+  const int LR = p.lift_res;                 // residues per CTA (4 or 8; all in one 32-residue group)
+  const int b = lid / p.lift_ctas, i0 = (lid - b * p.lift_ctas) * LR;
+  const int nres = min(LR, N - i0);
   const int RH = nres * H;
   const int PW = 2 * p.P38 + p.Q38;            // point row: [a' | b' | g'], each segment zero-padded
   const int nQ8 = p.Kq >> 3, nK8 = p.KHp >> 3, nV8 = p.VHp >> 3, nZ8 = p.Zp >> 3;
 
   float* wbt = reinterpret_cast<float*>(sh4);                // [H][Cz]  Wb^T / sqrt(3)
-  float* z1s = wbt + rup(H * Cz, 8);                         // [8][RC8]
-  float* qs = z1s + kLiftRes * p.RC8;                        // [8*H][D8]  q / sqrt(3D)
-  float* ks = qs + kLiftRes * H * p.D8;                      // [8*H][D8]
-  float* vs = ks + kLiftRes * H * p.D8;                      // [8*H][Dv8]
-  float* pts = vs + kLiftRes * H * p.Dv8;                    // [8*H][PW]  global point - o_G
-  float* frm = pts + kLiftRes * H * PW;                      // [8][12]  R (row-major), t - o_G
-  uint32_t* tab = reinterpret_cast<uint32_t*>(frm + kLiftRes * 12);   // chunk descriptors Q | K | V | Z
+  float* z1s = wbt + rup(H * Cz, 8);                         // [LR][RC8]
+  float* qs = z1s + LR * p.RC8;                              // [LR*H][D8]  q / sqrt(3D)
+  float* ks = qs + LR * H * p.D8;                            // [LR*H][D8]
+  float* vs = ks + LR * H * p.D8;                            // [LR*H][Dv8]
+  float* pts = vs + LR * H * p.Dv8;                          // [LR*H][PW]  global point - o_G
+  float* frm = pts + LR * H * PW;                            // [LR][12]  R (row-major), t
+  uint32_t* tab = reinterpret_cast<uint32_t*>(frm + LR * 12);   // chunk descriptors Q | K | V | Z
   __shared__ float s_gamma[64];
   __shared__ int s_valid[kLiftRes];
   __shared__ float4 s_orig;
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   // ---- phase 2: every point of every head, T_i(x) = R_i x + t_i relative to
   // the group origin (page "Invariant point attention (IPA)", Required
   // behavior: column-vector convention)
-  const float4 og = s_orig;                    // all kLiftRes residues share one group
+  const float4 og = s_orig;                    // all of the CTA's residues share one group
   auto apply = [&](const T* src, int npts, const FastDiv& fd_npts, int seg_off) {
     for (uint32_t e = threadIdx.x; e < (uint32_t)(RH * npts); e += blockDim.x) {
       const uint32_t rh = fd_npts.div(e), pt = e - rh * npts, r = p.fd_H.div(rh);
