@@ -78,7 +78,13 @@ typedef struct fipa_handle fipa_handle;
 /* Create a handle on CUDA device `device`.  `max_dims` may be NULL; if given,
  * later calls with any dim larger than it fail with FIPA_ERR_INVALID_ARG.
  * Allocates a few bytes of device memory for the status word (the only
- * allocation the library makes).  *out is NULL on failure. */
+ * allocation the library makes).  *out is NULL on failure.
+ * Environment read here, once per handle:
+ *   FIPA_WAIT_TIMEOUT_MS=<ms>  budget of every bounded device wait (default 2000)
+ *   FIPA_PAIR_SPLIT=0          bfloat16 mode: pair-bias operand as one fp16 half
+ *                              instead of hi + lo (faster; errors near the bf16
+ *                              tolerance, so off by default)
+ *   FIPA_TRACE_CTA=<n>         debug trace of one core CTA (see fipa_trace_copy) */
 fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims,
                         fipa_dtype dtype, int device);
 
