@@ -84,6 +84,11 @@ typedef struct fipa_handle fipa_handle;
  *   FIPA_PAIR_SPLIT=0          bfloat16 mode: pair-bias operand as one fp16 half
  *                              instead of hi + lo (faster; errors near the bf16
  *                              tolerance, so off by default)
+ *   FIPA_VALUE_BUFFER=0|1|2    bfloat16 mode: each key tile's value chunks land
+ *                              in a buffer of their own (the u lo chunks of the
+ *                              query tile then stream with the keys); 1 (default)
+ *                              from 8 key tiles per sample up, 2 wherever it
+ *                              fits, 0 never
  *   FIPA_TRACE_CTA=<n>         debug trace of one core CTA (see fipa_trace_copy) */
 fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims,
                         fipa_dtype dtype, int device);

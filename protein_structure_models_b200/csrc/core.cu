@@ -68,6 +68,7 @@ constexpr int kBarPVDone = 160;
 constexpr int kBarKtFull = 168;    // 2 x u64
 constexpr int kBarKtEmpty = 184;   // 2 x u64
 constexpr int kBarDrain = 200;
+constexpr int kBarVFull = 208;      // value buffer of the current key tile landed (value-buffer mode)
 constexpr int kOkBuf = 256;        // 2 x 4 key-group origins (float4)
 constexpr int kMisc = 384;         // tmem slot, abort flag, tile count
 constexpr int kKtBuf = 1024;       // 2 x 4 query groups x 128 keys per-key terms (floats)
@@ -241,14 +242,14 @@ struct EpiLayout {
 
 __device__ __forceinline__ EpiLayout epi_layout(const Plan& p, const void* z1) {
   EpiLayout e;
-  const uint32_t ring_end = (uint32_t)(p.nQc + p.nst) * kChunkBytes;
+  const uint32_t ring_end = (uint32_t)(p.nQres + (p.vbuf ? p.nVB : 0) + p.nst) * kChunkBytes;
   e.fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(z1) & 15) == 0;
   e.staged = e.fast_pair ? p.VHp : p.Ocols;
   e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.f32 ? 4 : 2));
   e.z1_stride = e.z1_row_bytes + 16;
   const uint32_t o_bytes = (uint32_t)kTile * (e.staged + 1) * 4;
   e.z1_smem = e.fast_pair && (e.z1_row_bytes & 15) == 0 &&
-              (uint32_t)kTile * e.z1_stride <= (uint32_t)p.nQc * kChunkBytes;
+              (uint32_t)kTile * e.z1_stride <= (uint32_t)p.nQres * kChunkBytes;
   e.o_off = e.z1_smem ? ((uint32_t)kTile * e.z1_stride + 1023u) & ~1023u : 0u;
   if (e.o_off + o_bytes > ring_end) { e.z1_smem = false; e.o_off = 0; }
   return e;
@@ -262,7 +263,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
 }
 
-template <bool SPLIT>
+// SPLIT: float32 inputs (3-way operands, P as hi + lo, exact point term).
+// VB: value-buffer mode (bfloat16 only): each key tile's value chunks [VH | Z]
+// land in a buffer of their own and the u lo chunks stream with the keys.
+template <bool SPLIT, bool VB>
 __global__ void __launch_bounds__(256, 1)
 fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKH,
                  const __grid_constant__ CUtensorMap tmVH, const __grid_constant__ CUtensorMap tmZ,
@@ -275,8 +279,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                         (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) == a.trace_cta;
   Tracer ttr{timeline ? a.trace + (size_t)2 * 2 * kTraceCap : nullptr, kTraceCap - 8};
   ttr.ev(40);
-  uint8_t* sQ = smem;
-  uint8_t* sRing = sQ + p.nQc * kChunkBytes;
+  uint8_t* sQ = smem;                                        // resident Qhat chunks
+  uint8_t* sV = sQ + p.nQres * kChunkBytes;                  // value buffer (value-buffer mode)
+  uint8_t* sRing = sV + (VB ? p.nVB : 0) * kChunkBytes;
   uint8_t* tail = sRing + p.nst * kChunkBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(tail + kBarFull);
   uint64_t* empty = reinterpret_cast<uint64_t*>(tail + kBarEmpty);
@@ -288,6 +293,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint64_t* kt_full = reinterpret_cast<uint64_t*>(tail + kBarKtFull);
   uint64_t* kt_empty = reinterpret_cast<uint64_t*>(tail + kBarKtEmpty);
   uint64_t* drain = reinterpret_cast<uint64_t*>(tail + kBarDrain);
+  uint64_t* v_full = reinterpret_cast<uint64_t*>(tail + kBarVFull);
   float* ktbuf = reinterpret_cast<float*>(tail + kKtBuf);
   float4* okbuf = reinterpret_cast<float4*>(tail + kOkBuf);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + kMisc);
@@ -313,6 +319,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     mbar_init(&kt_empty[0], 128);
     mbar_init(&kt_empty[1], 128);
     mbar_init(drain, 1);
+    mbar_init(v_full, 1);
     fence_mbar_init();
     *abort_flag = 0;
     // key tiles with a valid residue: the query's own tile first (it usually
@@ -352,8 +359,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tma_prefetch_desc(&tmKH);
       tma_prefetch_desc(&tmVH);
       tma_prefetch_desc(&tmZ);
-      mbar_arrive_expect_tx(q_full, (uint32_t)(p.nQc * kChunkBytes));
-      for (int c = 0; c < p.nQc; ++c) tma_load_3d(sQ + c * kChunkBytes, &tmQ, q_full, c * kChunk, qt * kTile, bh);
+      mbar_arrive_expect_tx(q_full, (uint32_t)(p.nQres * kChunkBytes));
+      for (int c = 0; c < p.nQres; ++c) tma_load_3d(sQ + c * kChunkBytes, &tmQ, q_full, c * kChunk, qt * kTile, bh);
       int st = 0;
       uint32_t ph = 0;
       bool ok = true;
@@ -370,7 +377,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (++st == p.nst) { st = 0; ph ^= 1u; }
       };
       auto push_qk = [&](int kt) {
-        for (int c = 0; c < p.nZ; ++c) push(&tmZ, c * kChunk, kt * kTile, b);
+        for (int c = 0; c < p.nZ; ++c) {
+          push(&tmZ, c * kChunk, kt * kTile, b);
+          // value-buffer mode: the u lo chunk that meets this z2 chunk
+          if (VB) push(&tmQ, (p.nKH + p.nZ + c) * kChunk, qt * kTile, bh);
+        }
         for (int c = 0; c < p.nKH; ++c) push(&tmKH, c * kChunk, kt * kTile, bh);
       };
       auto push_pv = [&](int kt) {
@@ -380,7 +391,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       push_qk(tiles[0]);
       for (int s = 0; s < nkt && ok; ++s) {
         if (s + 1 < nkt) push_qk(tiles[s + 1]);
-        push_pv(tiles[s]);
+        if (!VB) push_pv(tiles[s]);   // value-buffer mode: the MMA thread loads them
       }
       if (*abort_flag) {
         // wind down: let every load already issued land before the CTA exits
@@ -403,7 +414,100 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       uint32_t ph = 0;
       const uint32_t idS = idesc_f16(128, 128, 0, 0);
       const uint32_t sQa = smem_u32(sQ), sRa = smem_u32(sRing);
+      // value-buffer mode: the value chunks of key tile `kt` go to their own
+      // buffer; issued only once the P.V product that read it before is done
+      uint32_t v_issued = 0;
+      auto load_v = [&](int kt) {
+        mbar_arrive_expect_tx(v_full, (uint32_t)(p.nVB * kChunkBytes));
+        for (int c = 0; c < p.nVH; ++c) tma_load_3d(sV + c * kChunkBytes, &tmVH, v_full, c * kChunk, kt * kTile, bh);
+        for (int c = 0; c < p.nZV; ++c)
+          tma_load_3d(sV + (p.nVH + c) * kChunkBytes, &tmZ, v_full, c * kChunk, kt * kTile, b);
+        ++v_issued;
+      };
+      int v_pend = -1;                      // key-tile index s whose values wait for P.V(s-1)
+      auto poll_v = [&](bool block) -> bool {
+        if (v_pend < 0) return true;
+        const uint32_t par = (uint32_t)(v_pend - 1) & 1u;
+        if (block) {
+          if (!mbar_wait(pv_done, par, wc, 12)) return false;
+        } else if (!mbar_try_wait(pv_done, par)) {
+          return true;
+        }
+        load_v(tiles[v_pend]);
+        v_pend = -1;
+        return true;
+      };
+      // P.V(s) over the value buffer as a flat sequence of K-steps: runs of up
+      // to 4 64-column groups (N = 64 x run, groups 16 KB apart), 8 K-steps of
+      // 16 keys each.  (Issuing it in pieces between the QK^T(s+1) chunks was
+      // measured slower: the logits of the next tile then wait for it.)
+      auto mma_qk_vbuf = [&]() -> bool {
+        // ring order: per z2 chunk, [z2 | u lo]; the z2 chunk meets the resident
+        // u hi chunk and the streamed u lo chunk; then the head part.  The small
+        // pair terms accumulate before the large point terms.
+        for (int c = 0; c < p.nZ; ++c) {
+          tr.ev(11);
+          if (!mbar_wait(&full[st], ph, wc, 3)) return false;
+          tr.ev(12);
+          const int sz = st;
+          if (++st == p.nst) { st = 0; ph ^= 1u; }
+          tc_fence_after();
+          const uint32_t b0 = sRa + sz * kChunkBytes;
+          const uint32_t ah = sQa + (p.nKH + c) * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kTmemS, desc_kmajor_sw128(ah + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idS,
+                   (c | kk) != 0 ? 1u : 0u);
+          // the u lo half, as soon as its chunk has landed
+          tr.ev(11);
+          if (!mbar_wait(&full[st], ph, wc, 3)) return false;
+          tr.ev(12);
+          const int sl = st;
+          if (++st == p.nst) { st = 0; ph ^= 1u; }
+          tc_fence_after();
+          const uint32_t al = sRa + sl * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kTmemS, desc_kmajor_sw128(al + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idS, 1u);
+          tc_commit(&empty[sz]);
+          tc_commit(&empty[sl]);
+          if (!poll_v(false)) return false;
+        }
+        for (int c = 0; c < p.nKH; ++c) {
+          tr.ev(11);
+          if (!mbar_wait(&full[st], ph, wc, 3)) return false;
+          tr.ev(12);
+          tc_fence_after();
+          const uint32_t b0 = sRa + st * kChunkBytes, a0 = sQa + c * kChunkBytes;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kTmemS, desc_kmajor_sw128(a0 + kk * 32), desc_kmajor_sw128(b0 + kk * 32), idS, 1u);
+          tc_commit(&empty[st]);
+          if (++st == p.nst) { st = 0; ph ^= 1u; }
+        }
+        tc_commit(s_full);
+        tr.ev(17);
+        return true;
+      };
+      auto mma_pv_vbuf = [&](int s) -> bool {
+        if (!mbar_wait(v_full, (uint32_t)s & 1u, wc, 13)) return false;
+        tc_fence_after();
+        const uint32_t v0 = smem_u32(sV);
+        for (int c = 0; c < p.nVB; c += 4) {
+          const int run = p.nVB - c < 4 ? p.nVB - c : 4;
+          const uint32_t b0 = v0 + c * kChunkBytes;
+          const uint32_t idO = idesc_f16(128, 64 * run, 0, 1);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + (uint32_t)(p.tmemO + c * kChunk), tmem + kTmemP + kk * 8,
+                   desc_mnmajor_sw128(b0 + kk * 2048, kChunkBytes), idO, (s > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(pv_done);
+        tr.ev(18);
+        return true;
+      };
       auto mma_qk = [&]() -> bool {
+        if (VB) return mma_qk_vbuf();
         // key chunks in ring order: the pair part first (each z2 chunk meets nqz
         // Qhat chunks: u hi, u lo), the head part (scalar and point columns)
         // last, so the small pair terms accumulate before the large point terms
@@ -432,6 +536,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         return true;
       };
       auto mma_pv = [&](int s) -> bool {
+        if (VB) return mma_pv_vbuf(s);
         // value chunks in O-column order; up to 4 chunks in consecutive ring
         // slots form one MMA of N = 64 x run (MN-major B, groups 16 KB apart)
         const int nchunk = p.nVH + p.nZV;
@@ -463,6 +568,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tr.ev(18);
         return true;
       };
+      if (ok && VB) load_v(tiles[0]);
       if (ok) ok = mma_qk();
       for (int s = 0; ok && s < nkt; ++s) {
         if (s + 1 < nkt) {
@@ -472,15 +578,19 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tc_fence_after();
           if (!mma_qk()) break;
         }
+        if (VB && !poll_v(true)) break;   // this tile's values, if QK^T did not load them yet
         tr.ev(15);
         if (!mbar_wait(p_full, s & 1, wc, 6)) break;
         tr.ev(16);
         tc_fence_after();
         if (!mma_pv(s)) break;
+        if (VB && s + 1 < nkt) v_pend = s + 1;   // loads once P.V(s) has read the buffer
       }
-      // every MMA this thread issued has finished before the CTA tears down
+      // every MMA this thread issued has finished, and the last value load has
+      // landed, before the CTA tears down
       tc_commit(drain);
       drain_wait(drain, 0, a.timeout_ns);
+      if (v_issued > 0) drain_wait(v_full, (v_issued - 1) & 1u, a.timeout_ns);
     }
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ per-key terms
@@ -878,17 +988,11 @@ cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Ou
   a.status = ctl.status; a.timeout_ns = ctl.timeout_ns;
   a.trace = ctl.trace; a.trace_cta = ctl.trace_cta;
   dim3 grid(p.nT, p.H, p.B);
-  if (p.f32) {
-    auto kfn = fipa_core_kernel<true>;
-    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
-    if (e != cudaSuccess) return e;
-    kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);
-  } else {
-    auto kfn = fipa_core_kernel<false>;
-    cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
-    if (e != cudaSuccess) return e;
-    kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);
-  }
+  auto kfn = p.f32 ? fipa_core_kernel<true, false>
+                   : (p.vbuf ? fipa_core_kernel<false, true> : fipa_core_kernel<false, false>);
+  cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
+  if (e != cudaSuccess) return e;
+  kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);
   return cudaGetLastError();
 }
 

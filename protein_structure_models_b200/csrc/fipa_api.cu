@@ -37,6 +37,7 @@ struct fipa_handle {
   long long* d_trace = nullptr;
   int trace_cta = -1;
   int pair_split = 1;
+  int value_buffer = 1;
   // TMA descriptors of the last call: they depend only on the workspace
   // address and the dims, so a loop over the same buffers encodes them once
   struct MapCache {
@@ -91,7 +92,7 @@ fipa_status encode_rows(fipa_handle* h, CUtensorMap* m, const void* base, uint64
 int plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
   const char* why = "";
   int rc = fipa::make_plan(p, d->B, d->N, d->H, d->D, d->Dv, d->P, d->Q, d->Cz, d->R, d->Cout,
-                           h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split);
+                           h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split, h->value_buffer);
   if (rc != 0) h->last_error = why;
   return rc;
 }
@@ -150,6 +151,10 @@ FIPA_API fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims, f
   }
   h->encode = reinterpret_cast<EncodeTiledFn>(fn);
   if (const char* env = std::getenv("FIPA_PAIR_SPLIT")) h->pair_split = std::strtol(env, nullptr, 10) != 0;
+  if (const char* env = std::getenv("FIPA_VALUE_BUFFER")) {
+    const long v = std::strtol(env, nullptr, 10);
+    h->value_buffer = v <= 0 ? 0 : (v >= 2 ? 2 : 1);
+  }
   if (const char* env = std::getenv("FIPA_TRACE_CTA")) {
     h->trace_cta = (int)std::strtol(env, nullptr, 10);
     const size_t bytes = (size_t)4 * FIPA_TRACE_CAP * 2 * sizeof(long long);

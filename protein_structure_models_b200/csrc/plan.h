@@ -35,6 +35,7 @@ constexpr int kChunk = 64;       // fp16 columns per 128-byte swizzled chunk
 constexpr int kTmemS = 0;        // TMEM column of the logit tile S (128 fp32 columns)
 constexpr int kTmemP = 128;      // TMEM column of P (fp16 pairs: 64 columns, 128 when split)
 constexpr int kMaxQChunks = 10;  // resident Qhat tile <= 160 KB of shared memory
+constexpr int kVbufMinTiles = 8;  // key tiles from which the value-buffer mode pays
 constexpr int kMaxPts = 64;      // points per head handled by the prologue scratch
 constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
@@ -90,6 +91,13 @@ struct Plan {
   int Pcols;          // TMEM columns holding P (64, or 128 for hi+lo)
   int tmemO;          // TMEM column of the O accumulator
   int nst;            // shared-memory ring stages of the core kernel
+  // Value-buffer mode (bfloat16 inputs, when it fits): only QH and u hi of the
+  // Qhat tile stay resident, the u lo chunks stream through the ring with the
+  // key chunks, and each key tile's value chunks [VH | Z] land in a buffer of
+  // their own, so every P.V product runs over contiguous 64-column groups.
+  int vbuf;           // 1: value-buffer mode
+  int nQres;          // resident Qhat chunks (nQc, or nKH + nZ in value-buffer mode)
+  int nVB;            // value chunks per key tile (nVH + nZV); buffered in value-buffer mode
   size_t core_smem;   // dynamic shared memory of the core kernel
   size_t lift_smem;   // dynamic shared memory of the prologue lift kernel
   FastDiv fd_H, fd_P, fd_Q, fd_Cz;               // divisors of the lift kernel's index maps
@@ -119,9 +127,10 @@ struct Plan {
 
 // Returns 0 and fills `p`, or a nonzero reason code: 1 = bad dims, 2 = unsupported.
 // pair_split: 1 = pair-bias operand as fp16 hi + lo halves (bfloat16 inputs);
-// 0 = hi half only.
+// 0 = hi half only.  value_buffer: 1 = value-buffer mode where it fits and the
+// sample spans at least kVbufMinTiles key tiles, 2 = wherever it fits, 0 = off.
 static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, int Q, int Cz, int R,
-                            int Cout, int f32, const char** why, int pair_split = 1) {
+                            int Cout, int f32, const char** why, int pair_split = 1, int value_buffer = 1) {
   *why = "";
   if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || Dv <= 0 || P <= 0 || Q <= 0 || Cz <= 0 || R <= 0 ||
       Cout <= 0) {
@@ -171,14 +180,26 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   const size_t kp_bytes = p.geo_simt ? (size_t)2 * kTile * 3 * P * 4 : 0;
   const size_t fixed = 1024 + 5120 + 2 * kMaxTiles + kp_bytes;   // slack + tail (see core.cu)
   const size_t limit = 232448;  // 227 KB opt-in maximum per block on sm_100
-  size_t avail = limit - fixed - (size_t)p.nQc * 16384;
+  p.nVB = p.nVH + p.nZV;
+  p.vbuf = 0;
+  p.nQres = p.nQc;
+  // Measured on B200: 2-6% faster on the core from N = 2048 up; about 1% slower
+  // with two key tiles, where the serialised value loads are not hidden.
+  const bool vb_len = value_buffer == 2 || cdiv(N, kTile) >= kVbufMinTiles;
+  if (value_buffer && vb_len && p.nqz == 2 && !p.geo_simt) {
+    const int nres = p.nKH + p.nZ;
+    const long left = (long)limit - (long)fixed - (long)(nres + p.nVB) * 16384;
+    if (left >= 3 * 16384) { p.vbuf = 1; p.nQres = nres; }
+  }
+  size_t avail = limit - fixed - (size_t)(p.nQres + (p.vbuf ? p.nVB : 0)) * 16384;
   int nst = (int)(avail / 16384);
   if (nst > 8) nst = 8;
   if (nst < 3) { *why = "shared memory too small for the ring"; return 2; }
   p.nst = nst;
-  p.core_smem = fixed + (size_t)(p.nQc + nst) * 16384;
+  const int nchunks = p.nQres + (p.vbuf ? p.nVB : 0) + nst;   // Qhat, value buffer, ring
+  p.core_smem = fixed + (size_t)nchunks * 16384;
   if (p.core_smem < 120 * 1024) p.core_smem = 120 * 1024;   // one CTA per SM (TMEM is taken whole)
-  if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)(p.nQc + nst) * 16384) {
+  if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)nchunks * 16384) {
     *why = "value width too large for the epilogue staging"; return 2;
   }
   // prologue lift kernel: Wb^T, zero-padded z1 / q / k / v / point rows

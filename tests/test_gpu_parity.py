@@ -160,3 +160,24 @@ def test_validation_errors(handles):
     with pytest.raises(FipaError, match="UNSUPPORTED"):
         h.workspace_size(dict(B=1, N=8, H=1, D=1, Dv=1, P=65, Q=1, Cz=1, R=1, Cout=1))
     h.sync_status()
+
+
+# ------------------------------------------------------------------ core modes
+@pytest.mark.parametrize("mode", ["0", "2"])
+def test_value_buffer_modes(handles, monkeypatch, mode):
+    """The core's value-buffer mode (value chunks of each key tile in a buffer of
+    their own) is chosen by sample length; force it on for short samples and off
+    for a long one, so both paths stay parity-checked at every size class."""
+    from protein_structure_models_b200 import Fipa
+    monkeypatch.setenv("FIPA_VALUE_BUFFER", mode)
+    h = {"bf16": Fipa("bf16", 0)}
+    try:
+        check(h, workloads.make_inputs(workloads.workload(1)), "bf16")
+        for n in (129, 300):
+            check(h, _custom("bf16", 200 + n, N=n), "bf16")
+        n = 1024
+        inp = workloads.make_inputs(workloads.workload(f"3-{n}"))
+        rows = np.unique(np.concatenate([[0, 127, 128, n - 1], np.random.default_rng(7).choice(n, 60, replace=False)]))
+        check(h, inp, "bf16", rows=rows)
+    finally:
+        h["bf16"].close()
