@@ -7,9 +7,12 @@ A step is one full forward (prologue, fused attention core with the feature
 epilogue, output projection) over one batch of the workload's synthetic
 inputs, resident in HBM, replayed from a captured CUDA graph.  The L2 cache is flushed (a 256 MB write) between timed steps, outside
 the timed events.  Metric: query-key pairs per second, B*H*N^2 / t (padded
-N), summed over all ranks.  With N > 1 GPUs (torchrun) every rank runs its own
-replica of the workload on its own seed (weak scaling, no collective on the
-data path); the step time is the max over ranks.
+N), summed over all ranks.  With N > 1 GPUs (torchrun) every rank either runs
+its own replica of the workload on its own seed (weak scaling; the default for
+batched workloads), or, for a single-sample workload, lifts all keys of the
+same sample and computes its own contiguous range of query tiles through
+fipa_forward_rows (strong scaling; --shard).  No collective on the data path;
+the step time is the max over ranks.
 
 --impl reference times the CPU fp64 oracle on the host cores instead (each
 step: one sample of the batch), same metric and unit.
@@ -48,6 +51,10 @@ def parse_args():
                     help="0, 1, 2, 4 or 3-<N> (length sweep, N in 512..16384)")
     ap.add_argument("--impl", choices=("fipa", "reference"), default="fipa")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--shard", choices=("auto", "replicas", "rows"), default="auto",
+                    help="N > 1 GPUs: independent replicas (weak scaling) or the query rows of one "
+                         "batch split across ranks (strong scaling); auto = rows for a single-sample "
+                         "workload, replicas otherwise")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true",
@@ -234,6 +241,28 @@ def blas_threads():
 
 
 # ---------------------------------------------------------------- GPU arm
+def shard_mode(shard: str, wl, world: int) -> str:
+    """'rows' (every rank lifts all keys and computes its own query tiles of the
+    same inputs) or 'replicas' (every rank runs the whole workload on its own
+    seed)."""
+    if shard == "auto":
+        return "rows" if (wl.B == 1 and world > 1) else "replicas"
+    return shard
+
+
+def row_range(mask, rank: int, world: int):
+    """Query rows [r0, r1) of rank `rank` when the 128-row query tiles are split
+    into `world` contiguous ranges balanced by valid query rows (mask [B, N])."""
+    from protein_structure_models_b200.sharding import TILE, tile_rows, tile_shards
+    B, N = mask.shape
+    T = (N + TILE - 1) // TILE
+    weights = [int(mask[:, t * TILE:(t + 1) * TILE].sum()) for t in range(T)]
+    r0, r1 = tile_rows(tile_shards(weights, world)[rank], N)
+    if r0 >= r1:
+        raise ValueError(f"rank {rank} of {world} gets no query tile (N={N}): use fewer GPUs or --shard replicas")
+    return r0, r1
+
+
 def replica_seed(wl, rank: int) -> int:
     """Seed of rank `rank`'s replica: rank 0 runs the workload's own inputs."""
     return wl.seed + 1000 * rank
@@ -260,7 +289,9 @@ def run_fipa(args, wl, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    inp = workloads.make_inputs(wl, seed=replica_seed(wl, rank))
+    mode = shard_mode(args.shard, wl, world)
+    inp = workloads.make_inputs(wl, seed=wl.seed if mode == "rows" else replica_seed(wl, rank))
+    rows = row_range(inp["mask"], rank, world) if mode == "rows" else None
     d_in = to_device(inp, wl.dtype, dev)
     h = Fipa(wl.dtype, local_rank)
     dims = wl.dims()
@@ -271,7 +302,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     def forward():
-        h.forward(d_in, eps=inp["eps"], workspace=workspace, out=out, stream=stream)
+        h.forward(d_in, eps=inp["eps"], workspace=workspace, out=out, stream=stream, rows=rows)
 
     forward()                               # first call outside capture (one-time host setup)
     torch.cuda.synchronize()
@@ -282,7 +313,7 @@ def run_fipa(args, wl, rank, world, local_rank):
         cap = torch.cuda.Stream(dev)
         cap.wait_stream(stream)
         with torch.cuda.graph(g, stream=cap):
-            h.forward(d_in, eps=inp["eps"], workspace=workspace, out=out, stream=cap)
+            h.forward(d_in, eps=inp["eps"], workspace=workspace, out=out, stream=cap, rows=rows)
         torch.cuda.synchronize()
         return g
 
@@ -381,7 +412,7 @@ def run_fipa(args, wl, rank, world, local_rank):
         stream.wait_event(ev_in[j])
         if k >= 2:
             stream.wait_event(ev_out[j])        # download k-2 has read output j
-        h.forward(dev_in[j], eps=inp["eps"], workspace=workspace, out=dev_out[j], stream=stream)
+        h.forward(dev_in[j], eps=inp["eps"], workspace=workspace, out=dev_out[j], stream=stream, rows=rows)
         ev_fwd[j].record(stream)
         s_out.wait_event(ev_fwd[j])
         with torch.cuda.stream(s_out):
@@ -402,7 +433,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     e2e_ms = max_over_ranks(e2e_ms, dev)
     h.sync_status()
     h.close()
-    return dict(inp=inp, step_ms=step_ms_max, core_ms=core_ms, launches=launches,
+    return dict(inp=inp, mode=mode, step_ms=step_ms_max, core_ms=core_ms, launches=launches,
                 stage_ms={k: v / nb for k, v in stage_sum.items()}, clocks=clk,
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
 
@@ -451,7 +482,10 @@ def main_fipa(args, wl):
     padded, valid = pair_counts(wl, inp)
     fpp = flops_per_pair(wl)
     burst, sustained, hbm, src = measured_peaks()
-    value = padded * world / (r["step_ms"] / 1e3)
+    # replicas: every rank processed the whole workload; row shards: the ranks
+    # together processed it once
+    mult = world if r["mode"] == "replicas" else 1
+    value = padded * mult / (r["step_ms"] / 1e3)
     kernels = kernel_rooflines(wl, r["stage_ms"], valid, fpp, burst, hbm, src)
     stage_of = {"fipa_lift_kernel": "prologue", "fipa_core_kernel": "core", "fipa_out_proj_kernel": "out_proj"}
     dominant = max(kernels, key=lambda k: r["stage_ms"][stage_of[k]])
@@ -463,17 +497,20 @@ def main_fipa(args, wl):
                "sample": f"{done} whole sample(s) of the batch, all query rows, fp64 NumPy, {el:.1f} s"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True,
+        "scaling": "weak" if r["mode"] == "replicas" else "strong",
         "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-        "config": workload_config(wl, {"parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        "config": workload_config(wl, {"parallelism": "single GPU" if world == 1 else
+                                       (f"replicas x{world}" if r["mode"] == "replicas"
+                                        else f"query-row shards x{world}"),
                                        "l2": "flushed (256 MB write) between timed steps",
                                        "math": "fp16 tensor-core products, fp32 accumulate; bf16 inputs"}),
-        "valid_pairs_per_s": valid * world / (r["step_ms"] / 1e3),
+        "valid_pairs_per_s": valid * mult / (r["step_ms"] / 1e3),
         "stage_ms": r["stage_ms"],
         "roofline": roofline,
         "kernels": kernels,
         "cpu_baseline": cpu,
-        "e2e": {"value": padded * world / (r["e2e_ms"] / 1e3), "unit": UNIT,
+        "e2e": {"value": padded * mult / (r["e2e_ms"] / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "how": "public binding, pinned packed host buffers, one upload and one download per step, "
                        "two steps in flight (copies overlap the neighbouring forwards)"},

@@ -136,6 +136,32 @@ fipa_status fipa_forward(fipa_handle* h,
                          void* workspace, size_t workspace_bytes,
                          void* stream);
 
+/* The forward for query rows [row_begin, row_end) of every sample: the same
+ * arguments and outputs as fipa_forward, restricted to those rows.  Each
+ * output row depends on its own query and on all keys of its sample (page
+ * "Invariant point attention (IPA)", Required behavior: the softmax runs over
+ * every permitted key j of row i), so disjoint ranges, on one GPU or one per
+ * GPU, together give exactly the full forward, bit for bit.  Every key is still
+ * lifted (the prologue's O(N) work is repeated by each range); the fused core,
+ * the output projection and the optional attention output run only for the
+ * range's rows.  Rows outside the range are not written, in any output.
+ *   row_begin   multiple of 128 (the query tile), 0 <= row_begin < row_end
+ *   row_end     multiple of 128, or N; row_end <= N
+ * Anything else returns FIPA_ERR_INVALID_ARG before any launch. */
+fipa_status fipa_forward_rows(fipa_handle* h,
+                              const void* q, const void* k, const void* v,
+                              const void* q_pts, const void* k_pts, const void* v_pts,
+                              const void* rot, const void* trans,
+                              const void* z1, const void* z2, const void* Wb,
+                              const void* point_w_raw,
+                              const uint8_t* mask, const uint8_t* pair_mask,
+                              const void* w_out, const void* b_out, double eps,
+                              const fipa_dims* dims, int row_begin, int row_end,
+                              float* out_update, float* out_local_points,
+                              float* out_attention, float* out_lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream);
+
 /* Allocation-free forward.  No counterpart on the method's pages: this entry
  * point exists for callers that cannot allocate device memory where they call
  * the forward, e.g. code running while a CUDA graph is being captured (a

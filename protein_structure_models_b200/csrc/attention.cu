@@ -36,15 +36,16 @@ struct AttnArgs {
 __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
   const Plan& p = a.p;
   extern __shared__ float qs[];                 // [kRows][Kq]
-  const int i0 = blockIdx.x * kRows, h = blockIdx.y, b = blockIdx.z;
+  const int i0 = p.row0 + blockIdx.x * kRows, h = blockIdx.y, b = blockIdx.z;
   const int N = p.N, bh = b * p.H + h;
+  const int iend = p.row1;                      // rows of the forward's range (<= N)
   const float raw = p.f32 ? static_cast<const float*>(a.raw)[h]
                           : __bfloat162float(static_cast<const __nv_bfloat16*>(a.raw)[h]);
   const float g = point_weight(raw, p.P);
   for (int e = threadIdx.x; e < kRows * p.Kq; e += blockDim.x) {
     const int rr = e / p.Kq, c = e - rr * p.Kq;
     const int i = i0 + rr;
-    qs[e] = i < N ? __half2float(a.Q[((size_t)bh * N + i) * p.Kq + c]) : 0.f;
+    qs[e] = i < iend ? __half2float(a.Q[((size_t)bh * N + i) * p.Kq + c]) : 0.f;
   }
   __syncthreads();
   float M[kRows], l[kRows];
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
   for (int rr = 0; rr < kRows; ++rr) {
     const int i = i0 + rr;
     live[rr] = false;
-    if (i < N) {
+    if (i < iend) {
       const float2 st = a.stats[(size_t)bh * N + i];
       M[rr] = st.x; l[rr] = st.y;
       live[rr] = a.mask[(size_t)b * N + i] != 0 && st.y > 0.f;
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(128) fipa_attention_kernel(const AttnArgs a) {
     }
     for (int rr = 0; rr < kRows; ++rr) {
       const int i = i0 + rr;
-      if (i >= N) break;
+      if (i >= iend) break;
       float att = 0.f;
       bool permitted = live[rr] && kv.x != -INFINITY;
       if (permitted && a.pair_mask != nullptr) permitted = a.pair_mask[((size_t)b * N + i) * N + j] != 0;
@@ -124,7 +125,7 @@ cudaError_t launch_attention_dump(const Plan& p, const Inputs& in, const Work& w
   const size_t smem = (size_t)kRows * p.Kq * sizeof(float);
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_attention_kernel));
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((p.N + kRows - 1) / kRows), (unsigned)p.H, (unsigned)p.B);
+  dim3 grid((unsigned)((p.row1 - p.row0 + kRows - 1) / kRows), (unsigned)p.H, (unsigned)p.B);
   fipa_attention_kernel<<<grid, 128, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -303,7 +303,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   float* kpbuf = reinterpret_cast<float*>(tail + kKpBuf);          // [2][128][3P] (SPLIT only)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qt = blockIdx.x + p.row0 / kTile, h = blockIdx.y, b = blockIdx.z;
   const int bh = b * p.H + h;
   const int N = p.N, nT = p.nT;
 
@@ -987,7 +987,7 @@ cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Ou
   a.stats = w.stats; a.lse = out.lse;
   a.status = ctl.status; a.timeout_ns = ctl.timeout_ns;
   a.trace = ctl.trace; a.trace_cta = ctl.trace_cta;
-  dim3 grid(p.nT, p.H, p.B);
+  dim3 grid(cdiv(p.row1, kTile) - p.row0 / kTile, p.H, p.B);   // the query tiles of the row range
   auto kfn = p.f32 ? fipa_core_kernel<true, false>
                    : (p.vbuf ? fipa_core_kernel<false, true> : fipa_core_kernel<false, false>);
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));

@@ -28,6 +28,7 @@ struct ProjArgs {
   unsigned long long timeout_ns;
   long long* trace;   // debug timeline of one CTA (last slots of the MMA role's log), or null
   int trace_cta;
+  int tps;            // 0: tiles over the flattened B*N rows; else tiles per sample of the row range
 };
 
 // update[m, n] = sum_k feat[m, k] wT[n, k] + b_out[n], zero for empty rows.
@@ -49,7 +50,14 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tail + 256);
   int* abort_flag = reinterpret_cast<int*>(tail + 260);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kTile, n0 = blockIdx.y * ntile;
+  // output rows of this tile: [m0, min(m0 + 128, mlim))
+  int m0 = blockIdx.x * kTile, mlim = p.B * p.N;
+  if (a.tps > 0) {
+    const int bs = blockIdx.x / a.tps, t = blockIdx.x - bs * a.tps;
+    m0 = bs * p.N + p.row0 + t * kTile;
+    mlim = bs * p.N + p.row1;
+  }
+  const int n0 = blockIdx.y * ntile;
   const bool timeline = a.trace != nullptr && threadIdx.x == 0 &&
                         (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)) == a.trace_cta;
   Tracer ttr{timeline ? a.trace + (size_t)1 * 2 * kTraceCap : nullptr, kTraceCap - 8};
@@ -158,43 +166,58 @@ fipa_out_proj_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
   // shared memory, and writes them.  The second cluster barrier keeps every
   // tile alive until its readers are done.
   const int ks = p.gemm_ks;
+  // this lane's output columns: 4-column groups c4 = lane and lane + 32 (ntile
+  // <= 256); their bias is read before the barrier, off the reduce's path
+  const int nq = ntile / 4;
+  float bias[2][4];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int n = n0 + 4 * (lane + 32 * u) + e;
+      bias[u][e] = (lane + 32 * u < nq && n < p.Cout)
+                       ? (p.f32 ? static_cast<const float*>(a.b_out)[n]
+                                : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n]))
+                       : 0.f;
+    }
+  }
   cg::cluster_group cluster = cg::this_cluster();
   if (ks > 1) cluster.sync();
   else __syncthreads();
   ttr.ev(54);
   if (ok) {
-    const int M = p.B * p.N, nq = ntile / 4;
     const bool vec_out = (p.Cout & 3) == 0 && (reinterpret_cast<uintptr_t>(a.update) & 15) == 0;
     const int rows = (kTile + ks - 1) / ks, r0 = (int)blockIdx.z * rows, r1 = min(kTile, r0 + rows);
     for (int rr = r0 + warp; rr < r1; rr += 8) {
       const int m = m0 + rr;
-      if (m >= M) break;
+      if (m >= mlim) break;
       const bool keep = a.rowflag[m] != 0;
       float* urow = a.update + (size_t)m * p.Cout;
-      for (int c4 = lane; c4 < nq; c4 += 32) {
-        const int n = n0 + 4 * c4;
-        // all splits' loads in flight together, then added in split order
-        float4 t[8];
+      // every split's partial of both column groups in flight together, then
+      // added in split order (deterministic)
+      float4 t[2][8];
 #pragma unroll
-        for (int z = 0; z < 8; ++z) {
-          if (z < ks) {
-            const float* tz = ks > 1 ? cluster.map_shared_rank(stile, z) : stile;
-            t[z] = *reinterpret_cast<const float4*>(tz + (size_t)rr * sstride + 4 * c4);
-          }
+      for (int z = 0; z < 8; ++z) {
+        if (z < ks) {
+          const float* tz = (ks > 1 ? cluster.map_shared_rank(stile, z) : stile) + (size_t)rr * sstride;
+#pragma unroll
+          for (int u = 0; u < 2; ++u)
+            if (lane + 32 * u < nq) t[u][z] = *reinterpret_cast<const float4*>(tz + 4 * (lane + 32 * u));
         }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c4 = lane + 32 * u;
+        if (c4 >= nq) continue;
+        const int n = n0 + 4 * c4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int z = 0; z < 8; ++z) {
-          if (z < ks) { v.x += t[z].x; v.y += t[z].y; v.z += t[z].z; v.w += t[z].w; }
+          if (z < ks) { v.x += t[u][z].x; v.y += t[u][z].y; v.z += t[u][z].z; v.w += t[u][z].w; }
         }
         float w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float bo = n + e < p.Cout ? (p.f32 ? static_cast<const float*>(a.b_out)[n + e]
-                                                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.b_out)[n + e]))
-                                          : 0.f;
-          w[e] = keep ? w[e] + bo : 0.f;
-        }
+        for (int e = 0; e < 4; ++e) w[e] = keep ? w[e] + bias[u][e] : 0.f;
         if (vec_out && n + 4 <= p.Cout) {
           *reinterpret_cast<float4*>(urow + n) = make_float4(w[0], w[1], w[2], w[3]);
         } else {
@@ -403,13 +426,16 @@ static int resident_split(const Plan& p, int tiles) {
 
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl, cudaStream_t s) {
-  ProjArgs a{p, in.b_out, w.rowflag, out.update, ctl.status, ctl.timeout_ns, ctl.trace, ctl.trace_cta};
+  const bool full = p.row0 == 0 && p.row1 == p.N;
+  const int tps = full ? 0 : cdiv(p.row1 - p.row0, kTile);
+  ProjArgs a{p, in.b_out, w.rowflag, out.update, ctl.status, ctl.timeout_ns, ctl.trace, ctl.trace_cta, tps};
   const size_t BN = (size_t)p.B * p.N;
-  const unsigned mt = (unsigned)((BN + kTile - 1) / kTile), nt = (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out);
+  const unsigned mt = full ? (unsigned)((BN + kTile - 1) / kTile) : (unsigned)(p.B * tps);
+  const unsigned nt = (unsigned)(rup(p.Cout, p.ntile_out) / p.ntile_out);
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(fipa_out_proj_kernel));
   if (e != cudaSuccess) return e;
   const int nk = p.Kgp / kChunk;
-  if (p.gemm_ks == 1 && nt == 1) {
+  if (full && p.gemm_ks == 1 && nt == 1) {
     static int sm_count[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -424,7 +450,10 @@ cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, cons
       return cudaGetLastError();
     }
   }
-  const int ks = p.gemm_ks > 1 ? resident_split(p, (int)(mt * nt)) : 1;
+  // the split-K factor of the full forward, also for a row range, so that a
+  // range's rows add their K-splits exactly as the full forward does
+  const int mt_full = (int)((BN + kTile - 1) / kTile);
+  const int ks = p.gemm_ks > 1 ? resident_split(p, mt_full * (int)nt) : 1;
   a.p.gemm_nks = cdiv(nk, ks);
   a.p.gemm_ks = cdiv(nk, a.p.gemm_nks);
   // the split-K CTAs of one output tile form a cluster along z

@@ -295,13 +295,14 @@ FIPA_API fipa_status fipa_selftest_timeout(fipa_handle* h, unsigned timeout_ms, 
   return FIPA_OK;
 }
 
-FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
-                                  const void* k_pts, const void* v_pts, const void* rot, const void* trans,
-                                  const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
-                                  const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
-                                  const void* b_out, double eps, const fipa_dims* dims, float* out_update,
-                                  float* out_local_points, float* out_attention, float* out_lse, void* workspace,
-                                  size_t workspace_bytes, void* stream) {
+// The forward over query rows [row0, row1) of every sample (row1 < 0: N).
+static fipa_status forward_impl(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                const void* b_out, double eps, const fipa_dims* dims, int row0, int row1,
+                                float* out_update, float* out_local_points, float* out_attention, float* out_lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
   if (h == nullptr) return FIPA_ERR_INVALID_ARG;
   h->last_error.clear();
   if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
@@ -309,6 +310,13 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   const int rc = plan_for(h, dims, p);
   if (rc == 1) return FIPA_ERR_INVALID_ARG;
   if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  if (row1 < 0) row1 = p.N;
+  if (row0 < 0 || row0 >= row1 || row1 > p.N || row0 % fipa::kTile != 0 || (row1 % fipa::kTile != 0 && row1 != p.N))
+    return fail(h, FIPA_ERR_INVALID_ARG,
+                "row range must satisfy 0 <= row_begin < row_end <= N, row_begin a multiple of 128, "
+                "row_end a multiple of 128 or N");
+  p.row0 = row0;
+  p.row1 = row1;
   if (h->has_max) {
     const int* a = &dims->B;
     const int* m = &h->max_dims.B;
@@ -403,4 +411,29 @@ FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, 
   mark(4);
   h->timed_call = rec;
   return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_forward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                  const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                  const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                  const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                  const void* b_out, double eps, const fipa_dims* dims, float* out_update,
+                                  float* out_local_points, float* out_attention, float* out_lse, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  return forward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask, w_out,
+                      b_out, eps, dims, 0, -1, out_update, out_local_points, out_attention, out_lse, workspace,
+                      workspace_bytes, stream);
+}
+
+FIPA_API fipa_status fipa_forward_rows(fipa_handle* h, const void* q, const void* k, const void* v,
+                                       const void* q_pts, const void* k_pts, const void* v_pts, const void* rot,
+                                       const void* trans, const void* z1, const void* z2, const void* Wb,
+                                       const void* point_w_raw, const uint8_t* mask, const uint8_t* pair_mask,
+                                       const void* w_out, const void* b_out, double eps, const fipa_dims* dims,
+                                       int row_begin, int row_end, float* out_update, float* out_local_points,
+                                       float* out_attention, float* out_lse, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  return forward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask, w_out,
+                      b_out, eps, dims, row_begin, row_end, out_update, out_local_points, out_attention, out_lse,
+                      workspace, workspace_bytes, stream);
 }

@@ -74,6 +74,10 @@ struct Plan {
   int B, N, H, D, Dv, P, Q, Cz, R, Cout, F;
   int f32;            // 1: float32 inputs (hi/lo splits everywhere); 0: bfloat16 inputs
   int nT;             // tiles per sample
+  // query rows computed by this forward, the same range in every sample: row0
+  // a multiple of the 128-row tile, row1 a multiple of it or N (all keys are
+  // still lifted; rows outside the range are left untouched in the outputs)
+  int row0, row1;
   int nG;             // 32-residue origin groups per sample (4 per tile)
   int nsq;            // copies of the scalar q/k columns (1 or 3)
   int nsv;            // copies of the scalar v columns (1 or 2)
@@ -141,6 +145,8 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.F = H * (Dv + 4 * Q + Cz);
   p.f32 = f32 ? 1 : 0;
   p.nT = cdiv(N, kTile);
+  p.row0 = 0;
+  p.row1 = N;
   p.nG = 4 * p.nT;
   p.nsq = f32 ? 3 : 1;
   p.nsv = f32 ? 2 : 1;

@@ -58,6 +58,10 @@ def load_library():
                                                                 ctypes.POINTER(FipaDims)] \
         + [vp] * 4 + [vp, sz, vp]
     lib.fipa_forward.restype = c_int
+    lib.fipa_forward_rows.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double,
+                                                                     ctypes.POINTER(FipaDims), c_int, c_int] \
+        + [vp] * 4 + [vp, sz, vp]
+    lib.fipa_forward_rows.restype = c_int
     lib.fipa_sync_status.argtypes = [vp, vp]
     lib.fipa_sync_status.restype = c_int
     lib.fipa_selftest_timeout.argtypes = [vp, ctypes.c_uint, vp]
@@ -160,8 +164,12 @@ class Fipa:
 
     def forward(self, inp: dict, eps: float = 1e-8, want_attention: bool = False,
                 want_lse: bool = False, workspace: Optional[torch.Tensor] = None,
-                out: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None) -> dict:
-        """Run fipa_forward on torch tensors (see workloads.make_inputs for keys/layouts)."""
+                out: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None,
+                rows: Optional[tuple] = None) -> dict:
+        """Run fipa_forward on torch tensors (see workloads.make_inputs for keys/layouts).
+
+        rows=(row_begin, row_end): fipa_forward_rows, only those query rows of every
+        sample (the other rows of the outputs are left as they were)."""
         dev = torch.device("cuda", self.device)
         for k in INPUT_KEYS + ("w_out", "b_out"):
             t = inp[k]
@@ -186,12 +194,15 @@ class Fipa:
             workspace = torch.empty(self.workspace_size(dims), dtype=torch.uint8, device=dev)
         s = stream if stream is not None else torch.cuda.current_stream(dev)
         d = make_dims(**dims)
-        st = self.lib.fipa_forward(
-            self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(mask), _ptr(pair_mask),
-            _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d),
-            _ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("attention")),
-            _ptr(out.get("lse")), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
-            ctypes.c_void_p(s.cuda_stream))
+        head = (self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(mask), _ptr(pair_mask),
+                _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d))
+        tail = (_ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("attention")),
+                _ptr(out.get("lse")), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                ctypes.c_void_p(s.cuda_stream))
+        if rows is None:
+            st = self.lib.fipa_forward(*head, *tail)
+        else:
+            st = self.lib.fipa_forward_rows(*head, int(rows[0]), int(rows[1]), *tail)
         self._check(st)
         return out
 

@@ -44,7 +44,8 @@ def tile_shards(weights: Sequence[int], world: int) -> List[Tuple[int, int]]:
     """Split tiles 0..T-1 into `world` contiguous ranges with balanced total
     weight: range r ends at the first tile where the running weight reaches
     (r + 1) / world of the total.  Zero-weight tiles go with the range they
-    follow; with no weight at all the tiles are split evenly by count."""
+    follow; with no weight at all the tiles are split evenly by count.  With at
+    least as many tiles as ranks every range gets at least one tile."""
     T = len(weights)
     if world <= 0:
         raise ValueError("world must be > 0")
@@ -57,7 +58,11 @@ def tile_shards(weights: Sequence[int], world: int) -> List[Tuple[int, int]]:
             out.append((start, T))
             break
         goal = total * (r + 1) / world
-        while t < T and acc + weights[t] <= goal:
+        left = world - 1 - r                      # ranges after this one
+        while t < T - left and acc + weights[t] <= goal:
+            acc += weights[t]
+            t += 1
+        if t == start and t < T - left:           # never empty while tiles suffice
             acc += weights[t]
             t += 1
         out.append((start, t))

@@ -41,3 +41,39 @@ def test_prologue_bytes_matches_hand_count_for_protein_batch():
     reads = 2 * (BHN * (32 + 16 + 24 + 24) + BN * (12 + 512)) + BN
     writes = 2 * (BHN * (576 + 64 + 64) + BN * 256) + 32 * BHN
     assert bench.prologue_bytes(wl) == reads + writes
+
+
+def test_row_ranges_cover_every_row_once():
+    """--shard rows: the ranks' ranges are tile-aligned, disjoint and cover all
+    rows; the split follows the valid rows (a masked tail gets few ranks)."""
+    import workloads
+    for N, world, valid in [(4096, 8, 4096), (2048, 3, 2048), (1000, 4, 1000), (4096, 4, 1500)]:
+        mask = np.zeros((1, N), dtype=bool)
+        mask[0, :valid] = True
+        ranges = [bench.row_range(mask, r, world) for r in range(world)]
+        assert ranges[0][0] == 0 and ranges[-1][1] == N
+        for (a0, a1), (b0, b1) in zip(ranges, ranges[1:]):
+            assert a1 == b0 and a0 < a1
+        for r0, r1 in ranges:
+            assert r0 % 128 == 0 and (r1 % 128 == 0 or r1 == N)
+    # balanced by valid rows: with 1500 of 4096 valid, the first ranges are small
+    mask = np.zeros((1, 4096), dtype=bool)
+    mask[0, :1500] = True
+    ranges = [bench.row_range(mask, r, 4) for r in range(4)]
+    assert ranges[0][1] <= 512
+    assert bench.shard_mode("auto", workloads.workload("3-4096"), 4) == "rows"
+    assert bench.shard_mode("auto", workloads.workload(1), 4) == "replicas"
+    assert bench.shard_mode("auto", workloads.workload("3-4096"), 1) == "replicas"
+    assert bench.shard_mode("rows", workloads.workload(1), 1) == "rows"
+
+
+def test_row_range_rejects_more_ranks_than_tiles():
+    mask = np.ones((1, 256), dtype=bool)
+    assert [bench.row_range(mask, r, 2) for r in range(2)] == [(0, 128), (128, 256)]
+    raised = 0
+    for r in range(3):                       # 2 tiles, 3 ranks: one rank has nothing
+        try:
+            bench.row_range(mask, r, 3)
+        except ValueError:
+            raised += 1
+    assert raised == 1

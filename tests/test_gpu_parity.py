@@ -51,6 +51,7 @@ def test_workload0_tiny_f32(handles):
 def test_workload1_protein_batch(handles):
     inp = workloads.make_inputs(workloads.workload(1))
     check(handles, inp, "bf16")
+    check(handles, inp, "bf16", want_attention=False)   # as the benchmark runs it
 
 
 def test_workload2_rna_chain_sampled_rows(handles):
@@ -80,6 +81,7 @@ def test_workload4_short_chain_batch(handles):
     inp = workloads.make_inputs(workloads.workload(4))
     bsel = np.arange(0, 512, 16)           # 32 of the 512 samples, checked in full
     check(handles, inp, "bf16", bsel=bsel)
+    check(handles, inp, "bf16", bsel=bsel, want_attention=False)
 
 
 # ------------------------------------------------------------------ edge cases
@@ -110,6 +112,7 @@ def test_masks_and_empty_rows(handles, dtype):
     pm[0, :, 130:] = False                                       # a whole key tile blocked
     inp["pair_mask"] = pm
     check(handles, inp, dtype)
+    check(handles, inp, dtype, want_attention=False)
 
 
 def test_single_head_single_point(handles):
@@ -163,21 +166,81 @@ def test_validation_errors(handles):
 
 
 # ------------------------------------------------------------------ core modes
-@pytest.mark.parametrize("mode", ["0", "2"])
-def test_value_buffer_modes(handles, monkeypatch, mode):
+@pytest.mark.parametrize("env", [{"FIPA_VALUE_BUFFER": "0"}, {"FIPA_VALUE_BUFFER": "2"}],
+                         ids=["ring-only", "value-buffer"])
+def test_core_modes(handles, monkeypatch, env):
     """The core's value-buffer mode (value chunks of each key tile in a buffer of
-    their own) is chosen by sample length; force it on for short samples and off
-    for a long one, so both paths stay parity-checked at every size class."""
+    their own) is chosen by sample length; force it off and on for short and
+    long samples so both paths stay parity-checked at every size class."""
     from protein_structure_models_b200 import Fipa
-    monkeypatch.setenv("FIPA_VALUE_BUFFER", mode)
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
     h = {"bf16": Fipa("bf16", 0)}
     try:
-        check(h, workloads.make_inputs(workloads.workload(1)), "bf16")
-        for n in (129, 300):
-            check(h, _custom("bf16", 200 + n, N=n), "bf16")
+        # without the attention output, as the benchmark runs it
+        check(h, workloads.make_inputs(workloads.workload(1)), "bf16", want_attention=False)
+        for n in (1, 2, 129, 300):
+            check(h, _custom("bf16", 200 + n, N=n), "bf16", want_attention=False)
         n = 1024
         inp = workloads.make_inputs(workloads.workload(f"3-{n}"))
         rows = np.unique(np.concatenate([[0, 127, 128, n - 1], np.random.default_rng(7).choice(n, 60, replace=False)]))
-        check(h, inp, "bf16", rows=rows)
+        check(h, inp, "bf16", rows=rows, want_attention=False)
     finally:
         h["bf16"].close()
+
+
+# ------------------------------------------------------------------ query-row ranges
+def _row_range_case(handles, dtype, inp, world):
+    """fipa_forward_rows over the ranges of a `world`-way tile split (balanced by
+    valid tiles, as a multi-GPU run shards one sample) must rebuild the full
+    forward bit for bit; rows of no range stay untouched (NaN sentinel)."""
+    from protein_structure_models_b200.sharding import tile_rows, tile_shards
+    dev = to_device(inp, dtype)
+    h = handles[dtype]
+    full = h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True)
+    B, N = inp["mask"].shape
+    T = (N + 127) // 128
+    weights = [int(inp["mask"][:, t * 128:(t + 1) * 128].any()) for t in range(T)]
+    out = {k: torch.full_like(v, float("nan")) for k, v in full.items()}
+    ranges = [tile_rows(r, N) for r in tile_shards(weights, world)]
+    for r0, r1 in ranges:
+        if r0 < r1:
+            h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True, out=out, rows=(r0, r1))
+    h.sync_status()
+    torch.cuda.synchronize()
+    for k in full:
+        assert torch.equal(torch.nan_to_num(out[k], nan=7.0), torch.nan_to_num(full[k], nan=7.0)), k
+    # a single middle range: the rows outside it are not written
+    if N > 256:
+        part = {k: torch.full_like(v, float("nan")) for k, v in full.items()}
+        h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True, out=part, rows=(128, 256))
+        torch.cuda.synchronize()
+        for k, v in part.items():
+            rows_axis = 2 if k in ("attention", "lse") else 1
+            inside = v.narrow(rows_axis, 128, 128)
+            assert torch.equal(inside, full[k].narrow(rows_axis, 128, 128)), k
+            outside = torch.cat([v.narrow(rows_axis, 0, 128), v.narrow(rows_axis, 256, N - 256)], rows_axis)
+            assert torch.isnan(outside).all(), k
+
+
+def test_row_ranges_long_chain(handles):
+    _row_range_case(handles, "bf16", workloads.make_inputs(workloads.workload("3-1024")), 3)
+
+
+def test_row_ranges_ragged_batch(handles):
+    inp = _custom("bf16", 31, B=3, N=300)
+    inp["mask"][1, 200:] = False
+    _row_range_case(handles, "bf16", inp, 2)
+
+
+def test_row_ranges_f32(handles):
+    _row_range_case(handles, "f32", _custom("f32", 32, N=300), 2)
+
+
+def test_row_ranges_rejected(handles):
+    from protein_structure_models_b200.fipa import FipaError
+    inp = _custom("bf16", 33, N=300)
+    dev = to_device(inp, "bf16")
+    for rows in [(0, 0), (64, 256), (0, 200), (256, 128), (0, 301), (-128, 128)]:
+        with pytest.raises(FipaError):
+            handles["bf16"].forward(dev, eps=inp["eps"], rows=rows)
