@@ -371,10 +371,37 @@ __global__ void __launch_bounds__(kLiftThreads) fipa_lift_kernel(const PrologueA
   const uint32_t nthr = blockDim.x;
   // with the [u hi | u lo] pair layout a u-hi chunk also writes its lo
   // partner (the same products, the rounding residual instead of the value)
-  const uint32_t nQ8e = p.fd_nQ8e.d, uhi0 = (uint32_t)p.KHp >> 3, zch = (uint32_t)p.Zp >> 3;
+  const uint32_t uhi0 = (uint32_t)p.KHp >> 3, zch = (uint32_t)p.Zp >> 3;
   const bool pair_lo = p.nqz == 2;
+  // bfloat16 inputs with Cz a multiple of 8: the u chunks [u hi | u lo] of the
+  // Qhat rows get a loop of their own (no chunk table, no source dispatch);
+  // the table loop below then covers the head part only
+  const bool upath = !p.f32 && cz8;
+  if (upath) {
+    const uint32_t RCz8 = (uint32_t)RCz >> 3;
+    for (uint32_t e = threadIdx.x; e < (uint32_t)RH * zch; e += nthr) {
+      const uint32_t rh = p.fd_nZ8.div(e), j = e - rh * zch, r = p.fd_H.div(rh), h = rh - r * H;
+      float v[8];
+      if (j < RCz8 && s_valid[r] != 0) {
+        const uint32_t col = j << 3, cw = col - p.fd_Cz.div(col) * (uint32_t)Cz;   // channel c of column (r', c)
+        float w[8];
+        lds8(z1s + (size_t)r * p.RC8 + col, v);
+        lds8(wbt + (size_t)h * Cz + cw, w);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] *= w[t];
+      } else {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] = 0.f;
+      }
+      __half* urow = a.w.Q + (((size_t)b * H + h) * N + i0 + r) * p.Kq + p.KHp + ((size_t)j << 3);
+      stg8_half(urow, v, false);
+      if (pair_lo) stg8_half(urow + p.Zp, v, true);
+    }
+  }
+  const FastDiv& fdq = upath ? p.fd_nK8 : p.fd_nQ8e;
+  const uint32_t nQ8e = fdq.d;
   for (uint32_t e = threadIdx.x; e < (uint32_t)RH * nQ8e; e += nthr) {
-    const uint32_t rh = p.fd_nQ8e.div(e), c = e - rh * nQ8e, r = p.fd_H.div(rh), h = rh - r * H;
+    const uint32_t rh = fdq.div(e), c = e - rh * nQ8e, r = p.fd_H.div(rh), h = rh - r * H;
     const uint32_t d = tab[c];
     float v[8];
     chunk_values(d, s_valid[r] != 0, qs + (size_t)rh * p.D8, pts + (size_t)rh * PW, 2.f * s_gamma[h < 64 ? h : 63],
