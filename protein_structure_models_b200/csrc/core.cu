@@ -145,8 +145,8 @@ __device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col,
 
 // Features of residue bi for head h (page "Invariant point attention (IPA)",
 // Required behavior): scalar block; local point = R_i^T (sum_j a_ij g_j - t_i),
-// its length sqrt(|local|^2 + eps); pair block; all zero for an empty
-// neighbourhood.  orow = this row's O accumulator divided by l (staged in
+// its length sqrt(|local|^2 + eps); pair block.  For an empty neighbourhood
+// only the (zero) local points are written.  orow = this row's O accumulator divided by l (staged in
 // shared memory); (Gx,Gy,Gz) = sum_j a_ij o_G(j), the group-origin part of
 // the aggregated value points.  fblk = the (residue, head) block of the
 // projection operand, lp = the residue's local points of this head [Q][3].
@@ -156,11 +156,9 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
   const Plan& p = a.p;
   const int Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.Wh8;
   const int sc = 0, xc = Dv, pc = Dv + 4 * Q;
-  auto zero = [](int) { return 0.f; };
-  if (p.Wh8 > p.Wh) put_run(fblk, F, p.f32, p.Wh, p.Wh8 - p.Wh, zero);
   if (empty) {
-    put_run(fblk, F, p.f32, sc, Dv + 4 * Q, zero);
-    if (with_pair) put_run(fblk, F, p.f32, pc, Cz, zero);
+    // an empty neighbourhood: the local points are zero; the row's features
+    // are not written (the projection selects 0 for the row, whatever they hold)
     if (((3 * Q) & 3) == 0 && (reinterpret_cast<uintptr_t>(lp) & 15) == 0) {
       for (int e = 0; e < 3 * Q; e += 4) *reinterpret_cast<float4*>(lp + e) = make_float4(0.f, 0.f, 0.f, 0.f);
     } else {
@@ -168,6 +166,8 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
     }
     return;
   }
+  auto zero = [](int) { return 0.f; };
+  if (p.Wh8 > p.Wh) put_run(fblk, F, p.f32, p.Wh, p.Wh8 - p.Wh, zero);
   // scalar block
   put_run(fblk, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
   // points, 8 at a time in registers: aggregate (hi + lo halves + group-origin
@@ -956,7 +956,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv, acc[e]);
           }
         }
-        if (in_range) put_run32(frow, p.Wh8, p.f32, pcol + c0, acc);
+        if (in_range && !empty) put_run32(frow, p.Wh8, p.f32, pcol + c0, acc);
       }
     }
   }
