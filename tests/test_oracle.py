@@ -371,3 +371,100 @@ def test_planted_missing_point_scale_is_caught(monkeypatch):
     out = oracle.invariant_point_attention(act, par, masks, struct, eps=eps)
     a_self, _, _ = _worked_example_closed_form(3.0, eps)
     assert abs(out["attention"][0, 0, 0, 0] - a_self) > 0.05
+
+
+# --------------------------------------------------------------------------
+# the pair-bias term alone: closed form (logit bullet, pair_bias / sqrt(3))
+# --------------------------------------------------------------------------
+def _sigmoid(x):
+    return 1.0 / (1.0 + math.exp(-x))
+
+
+def _pair_bias_case(Wb_override=None):
+    """Two residues, identity frames at the origin, q = k = points = 0: the only
+    non-zero logit term is pair_bias / sqrt(3) (tests/golden/pair_bias_two_residues.json)."""
+    with open(os.path.join(GOLDEN, "pair_bias_two_residues.json")) as f:
+        fx = json.load(f)
+    B, N, H, D, Dv, P, Q, Cz, R = (fx[k] for k in ("B", "N", "H", "D", "Dv", "P", "Q", "Cz", "R"))
+    F = H * (Dv + 4 * Q + Cz)
+    inp = dict(q=np.zeros((B, N, H, D)), k=np.zeros((B, N, H, D)), v=np.ones((B, N, H, Dv)),
+               q_points=np.zeros((B, N, H, P, 3)), k_points=np.zeros((B, N, H, P, 3)),
+               v_points=np.zeros((B, N, H, Q, 3)),
+               rotation=np.tile(np.eye(3), (B, N, 1, 1)), translation=np.zeros((B, N, 3)),
+               z1=np.array(fx["z1_i_r_c"], float)[None], z2=np.array(fx["z2_j_r_c"], float)[None],
+               Wb=np.array(fx["Wb_c_h"], float) if Wb_override is None else Wb_override,
+               point_weight_raw=np.zeros(H), w_out=np.eye(F), b_out=np.zeros(F), eps=1e-8,
+               mask=np.ones((B, N), bool), pair_mask=None)
+    s3 = math.sqrt(3.0)
+    # hand-computed biases b_ij,h: b00 = (3, 1), b11 = (1, 4), b01 = b10 = 0
+    a = {(0, 0): _sigmoid(3 / s3), (1, 0): _sigmoid(1 / s3),      # (h, i): a[h][i][i]
+         (0, 1): _sigmoid(1 / s3), (1, 1): _sigmoid(4 / s3)}
+    pair_feat = np.array([[a[0, 0], 0.0, a[1, 0], 0.0],
+                          [0.0, 2 * a[0, 1], 0.0, 2 * a[1, 1]]])
+    return inp, a, pair_feat
+
+
+def test_pair_bias_closed_form_through_factors():
+    inp, a, pair_feat = _pair_bias_case()
+    for fn in (oracle.ipa_forward_dense, oracle.ipa_forward_factorised):
+        out = fn(inp, want_attention=True)
+        att = out["attention"][0]                          # [H, N, N]
+        for (h, i), val in a.items():
+            assert att[h, i, i] == pytest.approx(val, abs=1e-14)
+            assert att[h, i, 1 - i] == pytest.approx(1 - val, abs=1e-14)
+        np.testing.assert_allclose(out["update"][0][:, 10:14], pair_feat, atol=1e-14)
+
+
+def test_pair_bias_closed_form_through_page_signature():
+    """The same case through the page's dense signature: pair_bias [B,N,N,H] and
+    pair_values [B,N,N,Cz] written out by hand."""
+    inp, a, pair_feat = _pair_bias_case()
+    pb = np.zeros((1, 2, 2, 2))
+    pb[0, 0, 0] = [3.0, 1.0]
+    pb[0, 1, 1] = [1.0, 4.0]
+    pv = np.zeros((1, 2, 2, 2))
+    pv[0, 0, 0] = [1.0, 0.0]
+    pv[0, 1, 1] = [0.0, 2.0]
+    act = {k: inp[k] for k in ("q", "k", "v", "q_points", "k_points", "v_points")}
+    act.update(pair_bias=pb, pair_values=pv)
+    par = {k: inp[k] for k in ("point_weight_raw", "w_out", "b_out")}
+    out = oracle.invariant_point_attention(act, par, {"mask": inp["mask"], "pair_mask": None},
+                                           {"rotation": inp["rotation"], "translation": inp["translation"]},
+                                           eps=inp["eps"])
+    for (h, i), val in a.items():
+        assert out["attention"][0, h, i, i] == pytest.approx(val, abs=1e-14)
+    np.testing.assert_allclose(out["update"][0][:, 10:14], pair_feat, atol=1e-14)
+
+
+@pytest.mark.parametrize("plant", ["Wb transposed", "missing 1/sqrt(3)"])
+def test_pair_bias_pin_catches_planted_mistakes(plant):
+    """A transposed projection or a bias without its 1/sqrt(3) moves the
+    attention by far more than rounding (planted through the inputs)."""
+    Wb = np.array([[3.0, 1.0], [0.5, 2.0]])
+    wrong = Wb.T.copy() if plant == "Wb transposed" else Wb * math.sqrt(3.0)
+    inp, a, _ = _pair_bias_case(Wb_override=wrong)
+    att = oracle.ipa_forward_dense(inp, want_attention=True)["attention"][0]
+    worst = max(abs(att[h, i, i] - val) for (h, i), val in a.items())
+    assert worst > 0.05, worst
+
+
+# --------------------------------------------------------------------------
+# eps inside the output point lengths: worked example, length column of w_out
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("d", [0.0, 1.0, 3.0])
+def test_worked_example_lengths_with_eps(d):
+    """The page's worked example (eps = 1) with w_out picking the point-length
+    feature: update_i = sqrt(local_x_i^2 + eps), local_x = (1 + a_01 d, 1 - a_10 d)
+    and local y = z = 0.  At d = 0 the length is sqrt(2), not 1: eps is inside
+    the root ("used inside the OUTPUT point-length square root")."""
+    with open(os.path.join(GOLDEN, "worked_example_nearby_frames.json")) as f:
+        fx = json.load(f)
+    act, par, masks, struct, eps = _worked_example_inputs(fx, d)
+    assert eps == 1.0
+    par = dict(par, w_out=np.array([[0.0], [0.0], [0.0], [0.0], [1.0], [0.0]]))
+    out = oracle.invariant_point_attention(act, par, masks, struct, eps=eps)
+    _, _, loc_x = _worked_example_closed_form(d, eps)
+    want = [math.sqrt(x * x + 1.0) for x in loc_x]
+    np.testing.assert_allclose(out["update"][0, :, 0], want, atol=1e-13)
+    if d == 0.0:
+        np.testing.assert_allclose(out["update"][0, :, 0], math.sqrt(2.0), atol=1e-15)
