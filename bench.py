@@ -5,8 +5,12 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--impl fip
 
 A step is one full forward (prologue, fused attention core with the feature
 epilogue, output projection) over one batch of the workload's synthetic
-inputs, resident in HBM, replayed from a captured CUDA graph.  The L2 cache is flushed (a 256 MB write) between timed steps, outside
-the timed events.  Metric: query-key pairs per second, B*H*N^2 / t (padded
+inputs, resident in HBM, replayed from a captured CUDA graph.  The L2 cache
+is flushed (a 256 MB write) between timed steps, outside the timed events.
+The default workload is the longest chain of the length-scaling workload
+(B=1, N=16384), the largest that the configurations run on one GPU; its line
+also carries the whole length sweep (N = 512 ... 32768: time, peak device
+memory, fitted time exponent and memory line) under "sweep".  Metric: query-key pairs per second, B*H*N^2 / t (padded
 N), summed over all ranks.  With N > 1 GPUs (torchrun) every rank either runs
 its own replica of the workload on its own seed (weak scaling; the default for
 batched workloads), or, for a single-sample workload, lifts all keys of the
@@ -15,7 +19,8 @@ fipa_forward_rows (strong scaling; --shard).  No collective on the data path;
 the step time is the max over ranks.
 
 --impl reference times the CPU fp64 oracle on the host cores instead (each
-step: one sample of the batch), same metric and unit.
+step: one sample of the batch, or a block of its query rows for long chains),
+same metric and unit.
 """
 from __future__ import annotations
 
@@ -39,7 +44,7 @@ import workloads  # noqa: E402
 
 METRIC = "fused IPA fwd query-key pairs/sec (B·H·N²/s), % of B200 BF16 tensor peak"
 UNIT = "pairs/s"
-DEFAULT_WORKLOAD = "1"
+DEFAULT_WORKLOAD = "3-16384"
 
 
 def parse_args():
@@ -58,7 +63,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true",
-                    help="length sweep N=512..16384: time, peak memory, fitted exponents (JSON lines)")
+                    help="length sweep N=512..32768 only: time, peak memory, fitted exponents (JSON lines)")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave the length sweep out of the bench line (it runs after the timed steps)")
     return ap.parse_args()
 
 
@@ -209,26 +216,61 @@ def prologue_bytes(wl) -> int:
     return int(reads + writes)
 
 
-def out_proj_flops(wl) -> int:
-    """Algorithmic flops of update = features @ w_out over all B*N rows."""
+def live_rows(inp) -> int:
+    """Rows with a non-empty neighbourhood (mask_i and some permitted j): the
+    rows whose update the projection actually computes."""
+    mask = np.asarray(inp["mask"]).astype(bool)
+    pm = inp.get("pair_mask")
+    if pm is None:
+        return int(np.sum(mask & mask.any(axis=1, keepdims=True)))
+    permitted = mask[:, :, None] & mask[:, None, :] & np.asarray(pm).astype(bool)
+    return int(np.sum(permitted.any(axis=2)))
+
+
+def out_proj_flops(wl, rows: int) -> int:
+    """Algorithmic flops of update = features @ w_out over `rows` rows."""
     F = wl.H * (wl.Dv + 4 * wl.Q + wl.Cz)
-    return 2 * wl.B * wl.N * F * wl.Cout
+    return 2 * rows * F * wl.Cout
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
 def cpu_oracle_rate(wl, inp, seconds: float):
-    """Time the fp64 oracle on whole samples of the batch (all query rows) for
-    about `seconds`; returns (pairs/s in B*H*N^2 units, samples, threads, elapsed)."""
+    """Time the fp64 oracle on the host cores for about `seconds`.
+
+    Short samples: whole samples of the batch, all query rows.  When one sample
+    would take longer than `seconds` (the long chains), seeded query rows of
+    sample 0 against all N keys, in blocks of 128, at least 512 rows (each row
+    is exact on its own, so the rate carries over to the whole forward).
+    Returns (pairs/s in B*H*N^2 units, description of the sample)."""
     import oracle
-    done, t0 = 0, time.perf_counter()
+    rng = np.random.default_rng(wl.seed + 7)
+    t0 = time.perf_counter()
+    oracle.ipa_forward_dense(workloads.slice_batch(inp, [0]), rows=np.arange(min(16, wl.N)))
+    per_row = (time.perf_counter() - t0) / min(16, wl.N)
+    if per_row * wl.N <= seconds / 2:
+        done, t0 = 0, time.perf_counter()
+        while True:
+            oracle.ipa_forward_dense(workloads.slice_batch(inp, [done % wl.B]))
+            done += 1
+            el = time.perf_counter() - t0
+            if el >= seconds or done >= 10000:
+                break
+        return (done * wl.H * wl.N * wl.N / el,
+                f"{done} whole sample(s) of the batch, all query rows, fp64 NumPy, {el:.1f} s")
+    order = rng.permutation(wl.N)
+    one = workloads.slice_batch(inp, [0])
+    rows_done, t0 = 0, time.perf_counter()
     while True:
-        b = done % wl.B
-        oracle.ipa_forward_dense(workloads.slice_batch(inp, [b]))
-        done += 1
+        blk = np.sort(order[rows_done:rows_done + 128])
+        oracle.ipa_forward_dense(one, rows=blk)
+        rows_done += len(blk)
         el = time.perf_counter() - t0
-        if el >= seconds or done >= 10000:
+        if (el >= seconds and rows_done >= min(512, wl.N)) or rows_done >= wl.N:
             break
-    return done * wl.H * wl.N * wl.N / el, done, el
+    full = el * wl.B * wl.N / rows_done
+    return (rows_done * wl.H * wl.N / el,
+            f"{rows_done} seeded query rows of sample 0 against all {wl.N} keys, fp64 NumPy, {el:.1f} s "
+            f"(whole forward extrapolated: {full:.0f} s = {el:.1f} s x {wl.B * wl.N}/{rows_done} rows)")
 
 
 def blas_threads():
@@ -438,13 +480,13 @@ def run_fipa(args, wl, rank, world, local_rank):
                 e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
 
 
-def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src):
+def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src, rows):
     """Achieved rate of each timed kernel against its roofline; the time of a
     kernel is its stage's mean CUDA-event time inside the timed steps."""
     lift_s = stage_ms["prologue"] / 1e3
     core_s = stage_ms["core"] / 1e3
     proj_s = stage_ms["out_proj"] / 1e3
-    pb, pf, cf = prologue_bytes(wl), out_proj_flops(wl), valid * fpp
+    pb, pf, cf = prologue_bytes(wl), out_proj_flops(wl, rows), valid * fpp
     tensor_peak = f"{src} bf16 dense burst, {burst} TFLOP/s (fp16 operands run at the bf16 rate)"
     return {
         "fipa_lift_kernel": {
@@ -462,7 +504,8 @@ def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src):
         "fipa_out_proj_kernel": {
             "bound": "tensor", "achieved": pf / proj_s / 1e12, "peak": burst, "unit": "TFLOP/s",
             "frac": pf / proj_s / 1e12 / burst, "peak_source": tensor_peak,
-            "work": f"2*F*Cout flop x B*N rows = {pf} per launch; time = out_proj stage",
+            "work": f"2*F*Cout flop x {rows} rows with a non-empty neighbourhood = {pf} per launch; "
+                    f"time = out_proj stage",
             "traffic": profiled_traffic("fipa_out_proj_kernel", wl)},
     }
 
@@ -486,15 +529,14 @@ def main_fipa(args, wl):
     # together processed it once
     mult = world if r["mode"] == "replicas" else 1
     value = padded * mult / (r["step_ms"] / 1e3)
-    kernels = kernel_rooflines(wl, r["stage_ms"], valid, fpp, burst, hbm, src)
+    kernels = kernel_rooflines(wl, r["stage_ms"], valid, fpp, burst, hbm, src, live_rows(inp))
     stage_of = {"fipa_lift_kernel": "prologue", "fipa_core_kernel": "core", "fipa_out_proj_kernel": "out_proj"}
     dominant = max(kernels, key=lambda k: r["stage_ms"][stage_of[k]])
     roofline = dict(kernels[dominant], kernel=dominant)
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rate, done, el = cpu_oracle_rate(wl, inp, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{done} whole sample(s) of the batch, all query rows, fp64 NumPy, {el:.1f} s"}
+        rate, what = cpu_oracle_rate(wl, inp, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": what}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True,
@@ -517,6 +559,8 @@ def main_fipa(args, wl):
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    if world == 1 and wl.index == 3 and not args.no_sweep:
+        line["sweep"] = run_sweep(args.warmup)
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -527,22 +571,24 @@ def main_fipa(args, wl):
 def main_reference(args, wl):
     """The fp64 oracle on the host cores, same metric and unit.  Each step is one
     sample of the batch, or, when K whole samples would take more than about two
-    minutes, a block of that sample's query rows (every output row is exact on
-    its own); the block size comes from the time of whole samples in warm-up."""
+    minutes, a block of that sample's query rows against all keys (every output
+    row is exact on its own); the block size comes from the time of a small row
+    block in warm-up."""
     rank, world, _ = dist_info()
     if rank != 0:
         return
     import oracle
     inp = workloads.make_inputs(wl)
-    oracle.ipa_forward_dense(workloads.slice_batch(inp, [0]))      # first call: library start-up
-    t_full = []
+    probe = np.arange(min(16, wl.N))
+    oracle.ipa_forward_dense(workloads.slice_batch(inp, [0]), rows=probe)      # library start-up
+    t_row = []
     for k in range(max(1, args.warmup)):
         t0 = time.perf_counter()
-        oracle.ipa_forward_dense(workloads.slice_batch(inp, [k % wl.B]))
-        t_full.append(time.perf_counter() - t0)
-        if sum(t_full) > 20.0:
+        oracle.ipa_forward_dense(workloads.slice_batch(inp, [k % wl.B]), rows=probe)
+        t_row.append((time.perf_counter() - t0) / len(probe))
+        if sum(t_row) * len(probe) > 20.0:
             break
-    per_sample = float(np.median(t_full))
+    per_sample = float(np.median(t_row)) * wl.N
     budget = 120.0
     nrows = wl.N if args.steps * per_sample <= budget else max(1, int(wl.N * budget / (args.steps * per_sample)))
     t0 = time.perf_counter()
@@ -593,18 +639,20 @@ def fit_linear(ns, ys):
     return {"bytes_per_residue": float(a), "intercept_bytes": float(c), "r2": r2}
 
 
-def main_sweep(args):
-    """Length sweep: per N the graph-timed forward, and the peak device bytes
-    held by inputs, outputs and workspace (torch's peak counter, reset before
-    they are allocated); then the exponent of time vs N and the line of
-    memory vs N.  One JSON line per N, then one with the fits."""
+def run_sweep(warmup: int, emit=None) -> dict:
+    """Length sweep (the length-scaling workload, N = 512 ... 16384, plus the
+    32768 chain): per N the graph-timed forward (L2 flushed between steps) and
+    the peak device bytes held by inputs, outputs and workspace (torch's peak
+    counter, reset before they are allocated); then the least-squares exponent
+    of time vs N (all N, and N >= 2048) and the line of memory vs N.  `emit`,
+    if given, receives one dict per N."""
     import torch
     from protein_structure_models_b200 import Fipa
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    ns, ts, mems = [], [], []
-    for N in workloads.SWEEP_N:
+    ns, ts, mems, wss = [], [], [], []
+    for N in workloads.SWEEP_N + workloads.LONG_N:
         wl = workloads.workload(f"3-{N}")
         inp = workloads.make_inputs(wl)
         torch.cuda.synchronize()
@@ -625,7 +673,7 @@ def main_sweep(args):
             h.forward(d_in, eps=inp["eps"], workspace=ws, out=out, stream=cap)
         torch.cuda.synchronize()
         steps = max(5, min(200, int(2000 * 512 * 512 / N ** 2)))
-        for _ in range(max(3, args.warmup)):
+        for _ in range(max(3, warmup)):
             flush.zero_()
             graph.replay()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -640,16 +688,28 @@ def main_sweep(args):
         peak = torch.cuda.max_memory_allocated(dev) - base
         del graph
         h.close()
-        ns.append(N); ts.append(ms); mems.append(peak)
-        print(json.dumps({"sweep": "length", "N": N, "ms_per_forward": ms, "steps": steps,
-                          "pairs_per_s": wl.B * wl.H * N * N / (ms / 1e3), "peak_device_bytes": int(peak),
-                          "workspace_bytes": int(ws.numel())}), flush=True)
+        ns.append(N); ts.append(ms); mems.append(int(peak)); wss.append(int(ws.numel()))
+        if emit is not None:
+            emit({"sweep": "length", "N": N, "ms_per_forward": ms, "steps": steps,
+                  "pairs_per_s": wl.B * wl.H * N * N / (ms / 1e3), "peak_device_bytes": int(peak),
+                  "workspace_bytes": int(ws.numel())})
         del d_in, ws, out
         torch.cuda.empty_cache()
     big = [i for i, n in enumerate(ns) if n >= 2048]
-    print(json.dumps({"sweep": "length", "fit_time_all": fit_loglog(ns, ts),
-                      "fit_time_N_ge_2048": fit_loglog([ns[i] for i in big], [ts[i] for i in big]),
-                      "fit_memory": fit_linear(ns, mems)}), flush=True)
+    return {"N": ns, "ms_per_forward": ts, "peak_device_bytes": mems, "workspace_bytes": wss,
+            "fit_time_all": fit_loglog(ns, ts),
+            "fit_time_N_ge_2048": fit_loglog([ns[i] for i in big], [ts[i] for i in big]),
+            "fit_memory": fit_linear(ns, mems),
+            "how": "graph-replayed forward per N, median of CUDA-event steps, L2 flushed between steps; "
+                   "peak = torch max_memory_allocated of inputs + outputs + workspace"}
+
+
+def main_sweep(args):
+    """--sweep: one JSON line per N, then one with the fits."""
+    res = run_sweep(args.warmup, emit=lambda d: print(json.dumps(d), flush=True))
+    print(json.dumps({"sweep": "length", "fit_time_all": res["fit_time_all"],
+                      "fit_time_N_ge_2048": res["fit_time_N_ge_2048"],
+                      "fit_memory": res["fit_memory"]}), flush=True)
 
 
 def main():

@@ -164,26 +164,32 @@ fipa_status fipa_forward_rows(fipa_handle* h,
 
 /* Allocation-free forward.  No counterpart on the method's pages: this entry
  * point exists for callers that cannot allocate device memory where they call
- * the forward, e.g. code running while a CUDA graph is being captured (a
- * cudaMalloc there is forbidden or breaks the capture) or a plugin whose host
- * framework owns every device allocation through its own pool.  Such callers
+ * the forward: a plugin whose host framework owns every device allocation
+ * through its own pool and gives the plugin none, or a latency-bound caller
+ * that may not call cudaMalloc at run time (it can synchronise the device, and
+ * it can fail under memory pressure in the middle of a step).  Such callers
  * can create neither a workspace nor a handle (fipa_create allocates the
  * handle's status word), so this call takes neither.
  *
- * Scratch: one fixed device array of FIPA_NOALLOC_SCRATCH_BYTES inside the
- * library, held by every GPU that loads the library until the process exits.
- * Problems whose fipa_workspace_size exceeds it are rejected with
- * FIPA_ERR_WORKSPACE before anything is launched.  The call makes no
+ * Scratch: one fixed device array of FIPA_NOALLOC_SCRATCH_BYTES (32 MiB)
+ * inside the library, held by every GPU that loads the library until the
+ * process exits.  Problems whose fipa_workspace_size exceeds it are rejected
+ * with FIPA_ERR_WORKSPACE before anything is launched.  The call makes no
  * cudaMalloc / cudaFree and calls no allocating routine.
  *
- * Set-up: the first call on each device (the current device at call time)
- * looks up the array's device address with cudaGetSymbolAddress; make that
- * first call before any stream capture.
+ * Device: every pointer and `stream` must belong to the CURRENT device (the
+ * call looks up the scratch of the current device); q or out_update on
+ * another device returns FIPA_ERR_INVALID_ARG before any launch.
+ *
+ * Set-up: the first call on each device looks up the array's device address
+ * with cudaGetSymbolAddress and reads FIPA_WAIT_TIMEOUT_MS (as fipa_create
+ * does); a device that is not sm_100 returns FIPA_ERR_UNSUPPORTED there.
  *
  * Sharing: every call uses the same array and leaves its contents behind, so
  * calls whose kernels could overlap on the GPU (different streams without
  * ordering between them) race; order them on one stream or with events.
- * Nothing in the array needs clearing between calls.
+ * Nothing in the array needs clearing between calls: every kernel writes all
+ * of what a later kernel of the same call reads.
  *
  * Arguments and outputs are those of fipa_forward (no attention output); the
  * kernels run asynchronously on `stream`.  A bounded device-side wait that

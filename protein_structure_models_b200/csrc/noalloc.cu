@@ -1,18 +1,20 @@
 // noalloc.cu -- fipa_forward_noalloc: the fused IPA forward for callers that
 // cannot allocate device memory on their call path.
 //
-// Who needs it: code that runs while a CUDA graph is being captured (a
-// cudaMalloc there is forbidden or would break the capture), and plugins whose
-// host framework owns every device allocation through its own pool and gives
-// the plugin none.  Such callers cannot call cudaMalloc for a workspace, nor
-// fipa_create (which allocates the handle's status word).  This entry point
-// needs neither: its scratch is one fixed file-scope device array of
-// FIPA_NOALLOC_SCRATCH_BYTES, held by every GPU that loads this library until
-// the process exits, and its device status word is a file-scope variable too.
+// Who needs it: plugins whose host framework owns every device allocation
+// through its own pool and hands the plugin none, and latency-bound callers
+// that may not call cudaMalloc at run time (it can synchronise the device and
+// can fail under memory pressure in the middle of a step).  Such callers
+// cannot call cudaMalloc for a workspace, nor fipa_create (which allocates the
+// handle's status word).  This entry point needs neither: its scratch is one
+// fixed file-scope device array of FIPA_NOALLOC_SCRATCH_BYTES, held by every
+// GPU that loads this library until the process exits, and its device status
+// word is a file-scope variable too.
 //
 // The kernels and their launch order are those of fipa_forward; only where the
 // workspace comes from differs.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -38,6 +40,7 @@ struct DeviceState {
   bool ready = false;
   uint8_t* scratch = nullptr;   // device address of g_noalloc_scratch on this device
   int* status = nullptr;        // device address of g_noalloc_status on this device
+  unsigned long long timeout_ns = 2000000000ull;   // budget of every bounded device wait
 };
 std::mutex g_mu;
 DeviceState g_state[kMaxDevices];
@@ -50,6 +53,17 @@ fipa_status device_state(int dev, DeviceState** out) {
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& st = g_state[dev];
   if (!st.ready) {
+    // the kernels are built for sm_100a only
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FIPA_ERR_CUDA;
+    if (major != 10 || minor != 0) return FIPA_ERR_UNSUPPORTED;
+    // same wait budget as fipa_create: FIPA_WAIT_TIMEOUT_MS, read once per device
+    if (const char* env = std::getenv("FIPA_WAIT_TIMEOUT_MS")) {
+      const long ms = std::strtol(env, nullptr, 10);
+      if (ms > 0) st.timeout_ns = (unsigned long long)ms * 1000000ull;
+    }
     if (g_encode == nullptr) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -84,6 +98,18 @@ fipa_status encode(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// True when `p` is device (or managed) memory that device `dev` owns.  The
+// scratch address and the launches belong to the current device, so inputs on
+// another device are rejected before anything runs.
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();   // an unknown pointer leaves a (non-sticky) error behind: clear it
+    return false;
+  }
+  return (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) && a.device == dev;
+}
+
 }  // namespace
 
 FIPA_API fipa_status fipa_forward_noalloc(fipa_dtype dtype, const void* q, const void* k, const void* v,
@@ -115,6 +141,7 @@ FIPA_API fipa_status fipa_forward_noalloc(fipa_dtype dtype, const void* q, const
   DeviceState* ds = nullptr;
   fipa_status st = device_state(dev, &ds);
   if (st != FIPA_OK) return st;
+  if (!on_device(q, dev) || !on_device(out_update, dev)) return FIPA_ERR_INVALID_ARG;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = ds->scratch;
@@ -137,7 +164,7 @@ FIPA_API fipa_status fipa_forward_noalloc(fipa_dtype dtype, const void* q, const
   fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
                   w_out, b_out, (float)eps};
   fipa::Outputs out{out_update, out_local_points, nullptr, out_lse};
-  fipa::DeviceCtl ctl{ds->status, 2000000000ull, nullptr, -1};
+  fipa::DeviceCtl ctl{ds->status, ds->timeout_ns, nullptr, -1};
   const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
 
   CUtensorMap tmQ, tmKH, tmVH, tmZ, tmA, tmB;

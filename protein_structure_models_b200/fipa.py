@@ -233,12 +233,13 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 def forward_noalloc(inp: dict, eps: float = 1e-8, out: Optional[dict] = None,
                     stream: Optional[torch.cuda.Stream] = None) -> dict:
     """fipa_forward_noalloc: the forward without a handle or a workspace, for
-    callers that may not allocate device memory where they run it (inside a
-    CUDA graph capture, or under a host framework that owns all device
-    allocations).  Its scratch is a fixed 32 MiB device array inside the
-    library; `out`, if given, must hold preallocated "update" and
-    "local_points" (and optionally "lse") tensors, so this path allocates
-    nothing either."""
+    callers that may not allocate device memory where they run it (a plugin
+    whose host framework owns every device allocation, or a latency-bound
+    caller that may not call cudaMalloc mid-step).  Its scratch is a fixed
+    32 MiB device array inside the library; `out`, if given, must hold
+    preallocated "update" and "local_points" (and optionally "lse") tensors,
+    so this path allocates nothing either.  The call runs with the inputs'
+    device made current, as the C entry point requires."""
     lib = load_library()
     q = inp["q"]
     dtype = BF16 if q.dtype == torch.bfloat16 else F32
@@ -246,15 +247,17 @@ def forward_noalloc(inp: dict, eps: float = 1e-8, out: Optional[dict] = None,
     dims = dict(B=B, N=N, H=H, D=D, Dv=inp["v"].shape[-1], P=inp["q_points"].shape[3],
                 Q=inp["v_points"].shape[3], Cz=inp["z1"].shape[3], R=inp["z1"].shape[2],
                 Cout=inp["w_out"].shape[1])
-    if out is None:
-        out = {"update": torch.empty((B, N, dims["Cout"]), dtype=torch.float32, device=q.device),
-               "local_points": torch.empty((B, N, H, dims["Q"], 3), dtype=torch.float32, device=q.device)}
-    s = stream if stream is not None else torch.cuda.current_stream(q.device)
-    d = make_dims(**dims)
-    st = lib.fipa_forward_noalloc(
-        dtype, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]), _ptr(inp.get("pair_mask")),
-        _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d),
-        _ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("lse")), ctypes.c_void_p(s.cuda_stream))
+    with torch.cuda.device(q.device):
+        if out is None:
+            out = {"update": torch.empty((B, N, dims["Cout"]), dtype=torch.float32, device=q.device),
+                   "local_points": torch.empty((B, N, H, dims["Q"], 3), dtype=torch.float32, device=q.device)}
+        s = stream if stream is not None else torch.cuda.current_stream(q.device)
+        d = make_dims(**dims)
+        st = lib.fipa_forward_noalloc(
+            dtype, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]), _ptr(inp.get("pair_mask")),
+            _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d),
+            _ptr(out["update"]), _ptr(out["local_points"]), _ptr(out.get("lse")),
+            ctypes.c_void_p(s.cuda_stream))
     if st != FIPA_OK:
         raise FipaError(st, "fipa_forward_noalloc failed")
     return out

@@ -87,7 +87,7 @@ def test_reference_arm_prints_the_contract_line():
     import subprocess
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
-                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, timeout=300, cwd=root)
+                        "--steps", "2", "--warmup", "1", "--workload", "1"], capture_output=True, text=True, timeout=300, cwd=root)
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
     assert len(lines) == 1
@@ -98,3 +98,25 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"].startswith("protein-batch-bf16")
+
+
+def test_live_rows_and_projection_work():
+    """The projection's work is counted over rows with a non-empty
+    neighbourhood only (a masked row, or one whose pair_mask row is empty,
+    computes no update)."""
+    import workloads
+    wl = workloads.workload("1")
+    inp = workloads.make_inputs(wl)
+    live = int(inp["mask"].sum())
+    assert bench.live_rows(inp) == live
+    F = wl.H * (wl.Dv + 4 * wl.Q + wl.Cz)
+    assert bench.out_proj_flops(wl, live) == 2 * live * F * wl.Cout
+    w0 = workloads.workload(0)
+    inp0 = workloads.make_inputs(w0)          # one valid query has an all-false pair_mask row
+    assert bench.live_rows(inp0) == int(inp0["mask"].sum()) - 1
+
+
+def test_default_bench_workload_is_the_longest_single_gpu_chain():
+    import workloads
+    wl = workloads.workload(bench.DEFAULT_WORKLOAD)
+    assert (wl.B, wl.N) == (1, 16384) and wl.index == 3

@@ -69,7 +69,7 @@ def test_workload3_length_sweep(handles, n):
     check(handles, inp, "bf16", rows=rows, want_attention=(n <= 2048))
 
 
-@pytest.mark.parametrize("n", [8192, 16384])
+@pytest.mark.parametrize("n", [8192, 16384, 32768])
 def test_workload3_long_chains(handles, n):
     inp = workloads.make_inputs(workloads.workload(f"3-{n}"))
     rng = np.random.default_rng(n)
@@ -190,14 +190,15 @@ def test_core_modes(handles, monkeypatch, env):
 
 
 # ------------------------------------------------------------------ query-row ranges
-def _row_range_case(handles, dtype, inp, world):
+def _row_range_case(handles, dtype, inp, world, want_attention=True):
     """fipa_forward_rows over the ranges of a `world`-way tile split (balanced by
     valid tiles, as a multi-GPU run shards one sample) must rebuild the full
     forward bit for bit; rows of no range stay untouched (NaN sentinel)."""
     from protein_structure_models_b200.sharding import tile_rows, tile_shards
     dev = to_device(inp, dtype)
     h = handles[dtype]
-    full = h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True)
+    wa = want_attention
+    full = h.forward(dev, eps=inp["eps"], want_attention=wa, want_lse=True)
     B, N = inp["mask"].shape
     T = (N + 127) // 128
     weights = [int(inp["mask"][:, t * 128:(t + 1) * 128].any()) for t in range(T)]
@@ -205,7 +206,7 @@ def _row_range_case(handles, dtype, inp, world):
     ranges = [tile_rows(r, N) for r in tile_shards(weights, world)]
     for r0, r1 in ranges:
         if r0 < r1:
-            h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True, out=out, rows=(r0, r1))
+            h.forward(dev, eps=inp["eps"], want_attention=wa, want_lse=True, out=out, rows=(r0, r1))
     h.sync_status()
     torch.cuda.synchronize()
     for k in full:
@@ -213,7 +214,7 @@ def _row_range_case(handles, dtype, inp, world):
     # a single middle range: the rows outside it are not written
     if N > 256:
         part = {k: torch.full_like(v, float("nan")) for k, v in full.items()}
-        h.forward(dev, eps=inp["eps"], want_attention=True, want_lse=True, out=part, rows=(128, 256))
+        h.forward(dev, eps=inp["eps"], want_attention=wa, want_lse=True, out=part, rows=(128, 256))
         torch.cuda.synchronize()
         for k, v in part.items():
             rows_axis = 2 if k in ("attention", "lse") else 1
@@ -225,6 +226,14 @@ def _row_range_case(handles, dtype, inp, world):
 
 def test_row_ranges_long_chain(handles):
     _row_range_case(handles, "bf16", workloads.make_inputs(workloads.workload("3-1024")), 3)
+
+
+def test_row_ranges_32768_chain(handles):
+    """The 32768-residue chain (beyond the length sweep; the length that row
+    sharding across GPUs exists for) split 3 ways rebuilds the full forward bit
+    for bit.  Its parity with the oracle is test_workload3_long_chains[32768]."""
+    _row_range_case(handles, "bf16", workloads.make_inputs(workloads.workload("3-32768")), 3,
+                    want_attention=False)
 
 
 def test_row_ranges_ragged_batch(handles):

@@ -24,10 +24,13 @@ from typing import Optional
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "workload", "make_inputs", "round_to_dtype",
-           "random_rotations", "slice_batch", "SWEEP_N", "BASE_SEED"]
+           "random_rotations", "slice_batch", "SWEEP_N", "LONG_N", "BASE_SEED"]
 
 BASE_SEED = 20261202
 SWEEP_N = (512, 1024, 2048, 4096, 8192, 16384)
+# lengths beyond the sweep, same recipe: the single-chain length that row
+# sharding across GPUs exists for
+LONG_N = (32768,)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -89,7 +92,7 @@ def _w2():
 def _w3(n: int):
     return Workload(f"length-sweep-N{n}", 3, B=1, N=n, H=8, D=16, Dv=16, P=4, Q=8,
                     Cz=128, R=2, Cout=256, dtype="bf16", frames="walk", t_scale=3.8,
-                    sweep_index=SWEEP_N.index(n))
+                    sweep_index=(SWEEP_N + LONG_N).index(n))
 
 
 def _w4():
@@ -99,7 +102,7 @@ def _w4():
 
 
 WORKLOADS = {"0": _w0(), "1": _w1(), "2": _w2(), "4": _w4()}
-for _n in SWEEP_N:
+for _n in SWEEP_N + LONG_N:
     WORKLOADS[f"3-{_n}"] = _w3(_n)
 
 
