@@ -208,6 +208,63 @@ fipa_status fipa_forward_noalloc(fipa_dtype dtype,
                                  float* out_update, float* out_local_points, float* out_lse,
                                  void* stream);
 
+/* Gradients of the backward pass: float32 device buffers, each with the layout
+ * of the input it belongs to.  Every element is written. */
+typedef struct {
+  float* q;            /* [B,N,H,D]   */
+  float* k;            /* [B,N,H,D]   */
+  float* v;            /* [B,N,H,Dv]  */
+  float* q_pts;        /* [B,N,H,P,3] */
+  float* k_pts;        /* [B,N,H,P,3] */
+  float* v_pts;        /* [B,N,H,Q,3] */
+  float* rot;          /* [B,N,3,3]   */
+  float* trans;        /* [B,N,3]     */
+  float* z1;           /* [B,N,R,Cz]  */
+  float* z2;           /* [B,N,R,Cz]  */
+  float* Wb;           /* [Cz,H]      */
+  float* point_w_raw;  /* [H]         */
+  float* w_out;        /* [F,Cout]    */
+  float* b_out;        /* [Cout]      */
+} fipa_grads;
+
+/* Bytes of device workspace fipa_backward needs for `dims` (O(B*N): the
+ * forward's workspace plus the backward's per-residue buffers).  Pure host
+ * arithmetic.  FIPA_ERR_UNSUPPORTED for float32 inputs and for widths beyond
+ * the backward kernels' tensor-memory or shared-memory budget. */
+fipa_status fipa_backward_workspace_size(const fipa_handle* h, const fipa_dims* dims,
+                                         size_t* bytes);
+
+/* Backward pass (training).  The page "Invariant point attention (IPA)",
+ * section "Starter code", grades the full suite "including gradients"; this
+ * computes them: the gradient of <d_update, update> + <d_local_points,
+ * local_points> with respect to every floating input of fipa_forward (masks
+ * are not differentiated), written to `grads`.
+ *   inputs            exactly those of the fipa_forward call being differentiated
+ *   d_update          [B,N,Cout] float32 cotangent of update
+ *   d_local_points    [B,N,H,Q,3] float32 cotangent of local_points, or NULL (zero)
+ *   grads             float32 outputs (fipa_grads), caller-owned device buffers
+ *   workspace         >= fipa_backward_workspace_size() bytes, 256-byte aligned
+ * The call recomputes the forward it needs (the lift and the fused core, which
+ * also keeps the normalised aggregates of every row) inside the workspace, so
+ * it needs no state from an earlier fipa_forward.  Rows with an empty
+ * neighbourhood have constant (zero) outputs and pass no gradient back.
+ * bfloat16 inputs only (FIPA_ERR_UNSUPPORTED otherwise).  Allocates nothing,
+ * does not synchronise; kernels run on `stream`.  Deterministic: every sum is
+ * taken in a fixed order. */
+fipa_status fipa_backward(fipa_handle* h,
+                          const void* q, const void* k, const void* v,
+                          const void* q_pts, const void* k_pts, const void* v_pts,
+                          const void* rot, const void* trans,
+                          const void* z1, const void* z2, const void* Wb,
+                          const void* point_w_raw,
+                          const uint8_t* mask, const uint8_t* pair_mask,
+                          const void* w_out, const void* b_out, double eps,
+                          const fipa_dims* dims,
+                          const float* d_update, const float* d_local_points,
+                          const fipa_grads* grads,
+                          void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /* Wait for `stream`, then read and clear the handle's device status word.
  * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */

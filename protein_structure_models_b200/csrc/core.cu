@@ -55,6 +55,10 @@ struct CoreArgs {
   unsigned long long timeout_ns;
   long long* trace;
   int trace_cta;
+  // training recompute only (SAVE instantiation): normalised aggregates of
+  // every (residue, head), [B*N*H, Dv + 3Q + R*Cz] fp32 = [o_scalar | G (global
+  // value points, xyz per point) | U = sum_j a_ij z2_j], for the backward pass
+  float* osave;
 };
 
 // Shared-memory tail after the Qhat tile and the ring (byte offsets).
@@ -152,7 +156,7 @@ __device__ __forceinline__ void put_run32(__half* frow, int F, int f32, int col,
 // projection operand, lp = the residue's local points of this head [Q][3].
 __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* orow, float Gx, float Gy,
                                float Gz, bool with_pair, const float (&R)[9], const float (&t)[3], __half* fblk,
-                               float* lp) {
+                               float* lp, float* osv) {
   const Plan& p = a.p;
   const int Dv = p.Dv, Q = p.Q, Cz = p.Cz, F = p.Wh8;
   const int sc = 0, xc = Dv, pc = Dv + 4 * Q;
@@ -170,6 +174,8 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
   if (p.Wh8 > p.Wh) put_run(fblk, F, p.f32, p.Wh, p.Wh8 - p.Wh, zero);
   // scalar block
   put_run(fblk, F, p.f32, sc, Dv, [&](int d) { return p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d]; });
+  if (osv != nullptr)
+    for (int d = 0; d < Dv; ++d) osv[d] = p.f32 ? orow[d] + orow[p.Dv8 + d] : orow[d];
   // points, 8 at a time in registers: aggregate (hi + lo halves + group-origin
   // part), back into the query frame, lengths; then the x, y, z and length
   // feature runs and the local points straight from registers
@@ -186,6 +192,11 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
         const float gx = orow[gofs + 3 * q + 0] + orow[gofs + p.Q38 + 3 * q + 0] + Gx - t[0];
         const float gy = orow[gofs + 3 * q + 1] + orow[gofs + p.Q38 + 3 * q + 1] + Gy - t[1];
         const float gz = orow[gofs + 3 * q + 2] + orow[gofs + p.Q38 + 3 * q + 2] + Gz - t[2];
+        if (osv != nullptr) {
+          osv[Dv + 3 * q + 0] = gx + t[0];
+          osv[Dv + 3 * q + 1] = gy + t[1];
+          osv[Dv + 3 * q + 2] = gz + t[2];
+        }
         lx[u] = R[0] * gx + R[3] * gy + R[6] * gz;
         ly[u] = R[1] * gx + R[4] * gy + R[7] * gz;
         lz[u] = R[2] * gx + R[5] * gy + R[8] * gz;
@@ -215,6 +226,9 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
   // pair block through the factors (the tensor-memory path writes it otherwise)
   if (!with_pair) return;
   const int RCz = p.R * Cz;
+  if (osv != nullptr)
+    for (int rc = 0; rc < RCz; ++rc)
+      osv[Dv + 3 * Q + rc] = orow[p.VHp + rc] + (p.f32 ? orow[p.VHp + p.RC8 + rc] : 0.f);
   put_run(fblk, F, p.f32, pc, Cz, [&](int c) {
     float acc = 0.f;
     for (int rr = 0; rr < p.R; ++rr) {
@@ -266,7 +280,8 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 // SPLIT: float32 inputs (3-way operands, P as hi + lo, exact point term).
 // VB: value-buffer mode (bfloat16 only): each key tile's value chunks [VH | Z]
 // land in a buffer of their own and the u lo chunks stream with the keys.
-template <bool SPLIT, bool VB>
+// SAVE: also store the normalised aggregates of every row (training recompute).
+template <bool SPLIT, bool VB, bool SAVE>
 __global__ void __launch_bounds__(256, 1)
 fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKH,
                  const __grid_constant__ CUtensorMap tmVH, const __grid_constant__ CUtensorMap tmZ,
@@ -900,8 +915,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         if (h == 0) a.rowflag[bi] = empty ? 0 : 1;
         if (h == 0)
           for (int c = p.Kg; c < p.Kgp; ++c) a.feat[bi * p.Kgp + c] = __float2half_rn(0.f);
+        float* osv = SAVE ? a.osave + (bi * p.H + h) * (size_t)(p.Dv + 3 * p.Q + p.R * p.Cz) : nullptr;
         write_features(a, bi, empty, orow, rowW[0] * inv, rowW[1] * inv, rowW[2] * inv, !fast_pair, rowR, rowT,
-                       fblk, lp);
+                       fblk, lp, osv);
       }
       ttr.ev(46);
     } else if (fast_pair) {
@@ -954,6 +970,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             }
 #pragma unroll
             for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv, acc[e]);
+            if (SAVE) {
+              float* us = a.osave + (bi * p.H + h) * (size_t)(p.Dv + 3 * p.Q + RCz) + p.Dv + 3 * p.Q + rr * Cz + c0;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) us[e] = __uint_as_float(o[e]) * inv;
+            }
           }
         }
         if (in_range && !empty) put_run32(frow, p.Wh8, p.f32, pcol + c0, acc);
@@ -977,7 +998,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                         const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                        const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s) {
+                        const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s, float* osave) {
   CoreArgs a;
   a.p = p;
   a.kvec = w.kvec; a.qvec = w.qvec; a.QP = w.QP; a.KP = w.KP; a.orig = w.orig; a.flag = w.flag;
@@ -987,9 +1008,11 @@ cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Ou
   a.stats = w.stats; a.lse = out.lse;
   a.status = ctl.status; a.timeout_ns = ctl.timeout_ns;
   a.trace = ctl.trace; a.trace_cta = ctl.trace_cta;
+  a.osave = osave;
   dim3 grid(cdiv(p.row1, kTile) - p.row0 / kTile, p.H, p.B);   // the query tiles of the row range
-  auto kfn = p.f32 ? fipa_core_kernel<true, false>
-                   : (p.vbuf ? fipa_core_kernel<false, true> : fipa_core_kernel<false, false>);
+  auto kfn = p.f32 ? (osave ? fipa_core_kernel<true, false, true> : fipa_core_kernel<true, false, false>)
+                   : (p.vbuf ? (osave ? fipa_core_kernel<false, true, true> : fipa_core_kernel<false, true, false>)
+                             : (osave ? fipa_core_kernel<false, false, true> : fipa_core_kernel<false, false, false>));
   cudaError_t e = allow_max_smem(reinterpret_cast<const void*>(kfn));
   if (e != cudaSuccess) return e;
   kfn<<<grid, 256, p.core_smem, s>>>(tmQ, tmKH, tmVH, tmZ, a);

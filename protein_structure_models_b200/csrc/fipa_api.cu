@@ -46,6 +46,13 @@ struct fipa_handle {
     fipa_dims dims{};
     CUtensorMap Q, KH, VH, Z, A, B;
   } maps;
+  // the backward's dO map, cached the same way
+  struct BwdMapCache {
+    bool valid = false;
+    const void* ws = nullptr;
+    fipa_dims dims{};
+    CUtensorMap dO;
+  } bmaps;
 };
 
 namespace {
@@ -86,6 +93,52 @@ fipa_status encode_rows(fipa_handle* h, CUtensorMap* m, const void* base, uint64
   if (r != CUDA_SUCCESS)
     return fail(h, FIPA_ERR_CUDA, std::string("cuTensorMapEncodeTiled failed for ") + what + " (" +
                                       std::to_string((int)r) + ")");
+  return FIPA_OK;
+}
+
+// Work views of a workspace (plan.h layout).
+fipa::Work work_views(const Plan& p, void* workspace) {
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  fipa::Work w;
+  w.Q = reinterpret_cast<__half*>(ws + p.off_Q);
+  w.KH = reinterpret_cast<__half*>(ws + p.off_KH);
+  w.VH = reinterpret_cast<__half*>(ws + p.off_VH);
+  w.Z = reinterpret_cast<__half*>(ws + p.off_Z);
+  w.QP = reinterpret_cast<float*>(ws + p.off_QP);
+  w.KP = reinterpret_cast<float*>(ws + p.off_KP);
+  w.kvec = reinterpret_cast<float4*>(ws + p.off_kvec);
+  w.qvec = reinterpret_cast<float4*>(ws + p.off_qvec);
+  w.orig = reinterpret_cast<float4*>(ws + p.off_orig);
+  w.flag = reinterpret_cast<int*>(ws + p.off_flag);
+  w.stats = reinterpret_cast<float2*>(ws + p.off_stats);
+  w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
+  w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
+  w.rowflag = ws + p.off_rowflag;
+  return w;
+}
+
+// TMA descriptors of the lifted rows, the features and the prepared weights:
+// they depend only on the workspace address and the dims, so a loop over the
+// same buffers encodes them once.
+fipa_status ensure_maps(fipa_handle* h, const Plan& p, const fipa::Work& w, const void* workspace,
+                        const fipa_dims* dims) {
+  const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
+  fipa_handle::MapCache& mc = h->maps;
+  if (!mc.valid || mc.ws != workspace || std::memcmp(&mc.dims, dims, sizeof(fipa_dims)) != 0) {
+    mc.valid = false;
+    fipa_status st;
+    if ((st = encode_rows(h, &mc.Q, w.Q, p.Kq, N, BH, 128, 3, "Qhat")) != FIPA_OK) return st;
+    if ((st = encode_rows(h, &mc.KH, w.KH, p.KHp, N, BH, 128, 3, "Khat")) != FIPA_OK) return st;
+    if ((st = encode_rows(h, &mc.VH, w.VH, p.VHp, N, BH, 128, 3, "Vhat")) != FIPA_OK) return st;
+    if ((st = encode_rows(h, &mc.Z, w.Z, p.Zp, N, B, 128, 3, "Z")) != FIPA_OK) return st;
+    if ((st = encode_rows(h, &mc.A, w.feat, p.Kgp, B * N, 1, 128, 2, "features")) != FIPA_OK) return st;
+    if ((st = encode_rows(h, &mc.B, w.wT, p.Kgp, (uint64_t)fipa::rup(p.Cout, p.ntile_out), 1, p.ntile_out, 2,
+                          "w_out")) != FIPA_OK)
+      return st;
+    mc.ws = workspace;
+    mc.dims = *dims;
+    mc.valid = true;
+  }
   return FIPA_OK;
 }
 
@@ -343,46 +396,16 @@ static fipa_status forward_impl(fipa_handle* h, const void* q, const void* k, co
 
   DeviceGuard g(h->device);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  fipa::Work w;
-  w.Q = reinterpret_cast<__half*>(ws + p.off_Q);
-  w.KH = reinterpret_cast<__half*>(ws + p.off_KH);
-  w.VH = reinterpret_cast<__half*>(ws + p.off_VH);
-  w.Z = reinterpret_cast<__half*>(ws + p.off_Z);
-  w.QP = reinterpret_cast<float*>(ws + p.off_QP);
-  w.KP = reinterpret_cast<float*>(ws + p.off_KP);
-  w.kvec = reinterpret_cast<float4*>(ws + p.off_kvec);
-  w.qvec = reinterpret_cast<float4*>(ws + p.off_qvec);
-  w.orig = reinterpret_cast<float4*>(ws + p.off_orig);
-  w.flag = reinterpret_cast<int*>(ws + p.off_flag);
-  w.stats = reinterpret_cast<float2*>(ws + p.off_stats);
-  w.feat = reinterpret_cast<__half*>(ws + p.off_feat);
-  w.wT = reinterpret_cast<__half*>(ws + p.off_wT);
-  w.rowflag = ws + p.off_rowflag;
+  const fipa::Work w = work_views(p, workspace);
 
   fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
                   w_out, b_out, (float)eps};
   fipa::Outputs out{out_update, out_local_points, out_attention, out_lse};
   fipa::DeviceCtl ctl{h->d_status, h->timeout_ns, h->d_trace, h->trace_cta};
   if (h->d_trace != nullptr) cudaMemsetAsync(h->d_trace, 0xff, (size_t)4 * FIPA_TRACE_CAP * 2 * sizeof(long long), s);
-  const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
-
+  fipa_status mst = ensure_maps(h, p, w, workspace, dims);
+  if (mst != FIPA_OK) return mst;
   fipa_handle::MapCache& mc = h->maps;
-  if (!mc.valid || mc.ws != workspace || std::memcmp(&mc.dims, dims, sizeof(fipa_dims)) != 0) {
-    mc.valid = false;
-    fipa_status st;
-    if ((st = encode_rows(h, &mc.Q, w.Q, p.Kq, N, BH, 128, 3, "Qhat")) != FIPA_OK) return st;
-    if ((st = encode_rows(h, &mc.KH, w.KH, p.KHp, N, BH, 128, 3, "Khat")) != FIPA_OK) return st;
-    if ((st = encode_rows(h, &mc.VH, w.VH, p.VHp, N, BH, 128, 3, "Vhat")) != FIPA_OK) return st;
-    if ((st = encode_rows(h, &mc.Z, w.Z, p.Zp, N, B, 128, 3, "Z")) != FIPA_OK) return st;
-    if ((st = encode_rows(h, &mc.A, w.feat, p.Kgp, B * N, 1, 128, 2, "features")) != FIPA_OK) return st;
-    if ((st = encode_rows(h, &mc.B, w.wT, p.Kgp, (uint64_t)fipa::rup(p.Cout, p.ntile_out), 1, p.ntile_out, 2,
-                          "w_out")) != FIPA_OK)
-      return st;
-    mc.ws = workspace;
-    mc.dims = *dims;
-    mc.valid = true;
-  }
   const CUtensorMap &tmQ = mc.Q, &tmKH = mc.KH, &tmVH = mc.VH, &tmZ = mc.Z, &tmA = mc.A, &tmB = mc.B;
 
   cudaError_t e;
@@ -436,4 +459,102 @@ FIPA_API fipa_status fipa_forward_rows(fipa_handle* h, const void* q, const void
   return forward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask, w_out,
                       b_out, eps, dims, row_begin, row_end, out_update, out_local_points, out_attention, out_lse,
                       workspace, workspace_bytes, stream);
+}
+
+// ---------------------------------------------------------------- backward
+FIPA_API fipa_status fipa_backward_workspace_size(const fipa_handle* hc, const fipa_dims* dims, size_t* bytes) {
+  fipa_handle* h = const_cast<fipa_handle*>(hc);
+  if (h == nullptr || dims == nullptr || bytes == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "null argument");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  fipa::BwdPlan bp;
+  const char* why = "";
+  if (fipa::make_bwd_plan(bp, p, &why) != 0) return fail(h, FIPA_ERR_UNSUPPORTED, why);
+  *bytes = bp.total;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_backward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                   const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                   const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                   const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                   const void* b_out, double eps, const fipa_dims* dims, const float* d_update,
+                                   const float* d_local_points, const fipa_grads* grads, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
+  if (h->dtype != FIPA_BF16) return fail(h, FIPA_ERR_UNSUPPORTED, "the backward pass supports bfloat16 inputs only");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  if (h->has_max) {
+    const int* a = &dims->B;
+    const int* m = &h->max_dims.B;
+    for (int i = 0; i < 10; ++i)
+      if (a[i] > m[i]) return fail(h, FIPA_ERR_INVALID_ARG, "dims exceed the handle's max_dims");
+  }
+  fipa::BwdPlan bp;
+  const char* why = "";
+  if (fipa::make_bwd_plan(bp, p, &why) != 0) return fail(h, FIPA_ERR_UNSUPPORTED, why);
+  const void* req[] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, w_out, b_out};
+  const char* names[] = {"q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "Wb",
+                         "point_w_raw", "w_out", "b_out"};
+  for (int i = 0; i < 14; ++i) {
+    if (req[i] == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is NULL");
+    if (!aligned(req[i], 2)) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is misaligned");
+  }
+  if (mask == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "mask is NULL");
+  if (d_update == nullptr || !aligned(d_update, 4) || !aligned(d_local_points, 4))
+    return fail(h, FIPA_ERR_INVALID_ARG, "d_update is NULL or a cotangent is misaligned");
+  if (grads == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "grads is NULL");
+  float* const outs[] = {grads->q, grads->k, grads->v, grads->q_pts, grads->k_pts, grads->v_pts, grads->rot,
+                         grads->trans, grads->z1, grads->z2, grads->Wb, grads->point_w_raw, grads->w_out,
+                         grads->b_out};
+  for (int i = 0; i < 14; ++i)
+    if (outs[i] == nullptr || !aligned(outs[i], 4))
+      return fail(h, FIPA_ERR_INVALID_ARG, std::string("gradient of ") + names[i] + " is NULL or misaligned");
+  if (!(eps > 0.0) || !std::isfinite(eps)) return fail(h, FIPA_ERR_INVALID_ARG, "eps must be finite and > 0");
+  if (workspace == nullptr || workspace_bytes < bp.total)
+    return fail(h, FIPA_ERR_WORKSPACE, "backward workspace needs " + std::to_string(bp.total) + " bytes");
+  if (!aligned(workspace, 256)) return fail(h, FIPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+
+  DeviceGuard g(h->device);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const fipa::Work w = work_views(p, workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* osave = reinterpret_cast<float*>(ws + bp.off_osave);
+  fipa::Inputs in{q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
+                  w_out, b_out, (float)eps};
+  fipa::Outputs out{nullptr, reinterpret_cast<float*>(ws + bp.off_lp), nullptr, nullptr};
+  fipa::DeviceCtl ctl{h->d_status, h->timeout_ns, nullptr, -1};
+  fipa_status mst = ensure_maps(h, p, w, workspace, dims);
+  if (mst != FIPA_OK) return mst;
+  fipa_handle::BwdMapCache& bm = h->bmaps;
+  if (!bm.valid || bm.ws != workspace || std::memcmp(&bm.dims, dims, sizeof(fipa_dims)) != 0) {
+    bm.valid = false;
+    if ((mst = encode_rows(h, &bm.dO, ws + bp.off_dO, bp.Vw, (uint64_t)p.N, (uint64_t)p.B * p.H, 128, 3, "dO")) !=
+        FIPA_OK)
+      return mst;
+    bm.ws = workspace;
+    bm.dims = *dims;
+    bm.valid = true;
+  }
+  const fipa_handle::MapCache& mc = h->maps;
+  fipa::BwdIO io{d_update, d_local_points,
+                 fipa::BwdGrads{grads->q, grads->k, grads->v, grads->q_pts, grads->k_pts, grads->v_pts, grads->rot,
+                                grads->trans, grads->z1, grads->z2, grads->Wb, grads->point_w_raw, grads->w_out,
+                                grads->b_out},
+                 ws};
+  cudaError_t e;
+  // recompute: the lift, and the core saving the normalised aggregates
+  if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
+  if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
+    return cuda_fail(h, "core launch", e);
+  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, ctl, s)) != cudaSuccess)
+    return cuda_fail(h, "backward launch", e);
+  return FIPA_OK;
 }

@@ -10,6 +10,7 @@
 #include <mutex>
 #include <utility>
 
+#include "bwd_plan.h"
 #include "plan.h"
 
 namespace fipa {
@@ -88,14 +89,32 @@ struct Tracer {
 
 // Launchers return the cudaError_t of the launch.
 cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cudaStream_t s);
+// osave: null for the forward; the backward's recompute passes its buffer of
+// normalised aggregates (see CoreArgs in core.cu).
 cudaError_t launch_core(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                         const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                        const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s);
+                        const CUtensorMap& tmZ, const DeviceCtl& ctl, cudaStream_t s, float* osave = nullptr);
 cudaError_t launch_out_proj(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                             const CUtensorMap& tmA, const CUtensorMap& tmB, const DeviceCtl& ctl,
                             cudaStream_t s);
 cudaError_t launch_attention_dump(const Plan& p, const Inputs& in, const Work& w, const Outputs& out,
                                   cudaStream_t s);
+
+// Gradient outputs of the backward pass (float32, layouts of the inputs).
+struct BwdGrads {
+  float *q, *k, *v, *q_pts, *k_pts, *v_pts, *rot, *trans, *z1, *z2, *Wb, *raw, *w_out, *b_out;
+};
+struct BwdIO {
+  const float* d_update;   // [B,N,Cout] cotangent of update
+  const float* d_local;    // [B,N,H,Q,3] cotangent of local_points, or null (zero)
+  BwdGrads g;
+  uint8_t* ws;             // workspace base (backward regions at the BwdPlan offsets)
+};
+// The backward kernels after the recompute (lift, and the core with the
+// aggregates saved at the BwdPlan's osave offset).
+cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
+                            const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
+                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s);
 
 // Per-head distance weight 1/2 softplus(raw) sqrt(2/(27P)), softplus without overflow.
 __device__ __forceinline__ float point_weight(float raw, int P) {

@@ -27,6 +27,14 @@ class FipaDims(ctypes.Structure):
     _fields_ = [(f, ctypes.c_int) for f in DIM_FIELDS]
 
 
+GRAD_FIELDS = ("q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "Wb", "point_w_raw",
+               "w_out", "b_out")
+
+
+class FipaGrads(ctypes.Structure):
+    _fields_ = [(f, ctypes.c_void_p) for f in GRAD_FIELDS]
+
+
 class FipaError(RuntimeError):
     def __init__(self, status: int, message: str):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
@@ -82,6 +90,11 @@ def load_library():
                                                                          ctypes.POINTER(FipaDims)] \
         + [vp] * 3 + [vp]
     lib.fipa_forward_noalloc.restype = c_int
+    lib.fipa_backward_workspace_size.argtypes = [vp, ctypes.POINTER(FipaDims), ctypes.POINTER(sz)]
+    lib.fipa_backward_workspace_size.restype = c_int
+    lib.fipa_backward.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double, ctypes.POINTER(FipaDims)] \
+        + [vp, vp, ctypes.POINTER(FipaGrads), vp, sz, vp]
+    lib.fipa_backward.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -205,6 +218,47 @@ class Fipa:
             st = self.lib.fipa_forward_rows(*head, int(rows[0]), int(rows[1]), *tail)
         self._check(st)
         return out
+
+    # input key of each gradient (fipa_grads field -> workloads key)
+    GRAD_KEYS = {"q": "q", "k": "k", "v": "v", "q_pts": "q_points", "k_pts": "k_points", "v_pts": "v_points",
+                 "rot": "rotation", "trans": "translation", "z1": "z1", "z2": "z2", "Wb": "Wb",
+                 "point_w_raw": "point_weight_raw", "w_out": "w_out", "b_out": "b_out"}
+
+    def backward_workspace_size(self, dims: dict) -> int:
+        d = make_dims(**dims)
+        n = ctypes.c_size_t()
+        self._check(self.lib.fipa_backward_workspace_size(self.handle, ctypes.byref(d), ctypes.byref(n)))
+        return int(n.value)
+
+    def backward(self, inp: dict, d_update: torch.Tensor, d_local: Optional[torch.Tensor] = None,
+                 eps: float = 1e-8, workspace: Optional[torch.Tensor] = None, grads: Optional[dict] = None,
+                 stream: Optional[torch.cuda.Stream] = None) -> dict:
+        """fipa_backward: float32 gradients of <d_update, update> + <d_local, local_points>
+        for every floating input, keyed like the inputs (see workloads.make_inputs)."""
+        dev = torch.device("cuda", self.device)
+        for k in INPUT_KEYS + ("w_out", "b_out"):
+            t = inp[k]
+            if t.dtype != self.torch_dtype or t.device != dev or not t.is_contiguous():
+                raise ValueError(f"{k}: need a contiguous {self.torch_dtype} tensor on {dev}")
+        for name, t in (("d_update", d_update), ("d_local", d_local)):
+            if t is not None and (t.dtype != torch.float32 or t.device != dev or not t.is_contiguous()):
+                raise ValueError(f"{name}: need a contiguous float32 tensor on {dev}")
+        dims = self.dims_of(inp)
+        if grads is None:
+            grads = {key: torch.empty(inp[key].shape, dtype=torch.float32, device=dev)
+                     for key in self.GRAD_KEYS.values()}
+        if workspace is None:
+            workspace = torch.empty(self.backward_workspace_size(dims), dtype=torch.uint8, device=dev)
+        gs = FipaGrads(*[grads[self.GRAD_KEYS[f]].data_ptr() for f in GRAD_FIELDS])
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        d = make_dims(**dims)
+        st = self.lib.fipa_backward(self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]),
+                                    _ptr(inp.get("pair_mask")), _ptr(inp["w_out"]), _ptr(inp["b_out"]),
+                                    float(eps), ctypes.byref(d), _ptr(d_update), _ptr(d_local), ctypes.byref(gs),
+                                    _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+                                    ctypes.c_void_p(s.cuda_stream))
+        self._check(st)
+        return grads
 
     STAGES = ("prologue", "core", "out_proj", "attention")
 

@@ -1,0 +1,138 @@
+"""The CUDA backward pass (fipa_backward, through the C ABI) against the fp64
+backward oracle (oracle/backward.py: the vector-Jacobian product of the page's
+forward, "Invariant point attention (IPA)", Required behavior; the page's
+"Starter code" section grades the suite "including gradients").
+
+Tolerance (bfloat16 inputs; the derivation is in the design notes): for every
+gradient tensor, max |g - g_ref| <= GRAD_TOL * max |g_ref|, GRAD_TOL = 1e-2.
+The fp16 operands of the recomputed products and of dS carry 2^-11 relative
+rounding each; dS = P (dP - D) loses up to a few bits where dP is close to D;
+1e-2 allows a 20x amplification of one fp16 rounding.  Residues with mask 0
+pass no gradient at all, so theirs must be exactly zero."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import backward as bw
+from parity_util import to_device
+
+pytestmark = pytest.mark.gpu
+
+GRAD_TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def handle():
+    from protein_structure_models_b200 import Fipa, build
+    build.build()
+    h = Fipa("bf16", 0)
+    yield h
+    h.close()
+
+
+def _cotangents(inp, seed):
+    rng = np.random.default_rng(seed)
+    B, N, H = inp["q"].shape[:3]
+    Q, Cout = inp["v_points"].shape[3], inp["w_out"].shape[1]
+    return rng.standard_normal((B, N, Cout)), rng.standard_normal((B, N, H, Q, 3))
+
+
+def run_backward(handle, inp, du, dl):
+    dev = to_device(inp, "bf16")
+    d_update = torch.from_numpy(du).float().cuda().contiguous()
+    d_local = torch.from_numpy(dl).float().cuda().contiguous()
+    g = handle.backward(dev, d_update, d_local, eps=inp["eps"])
+    handle.sync_status()
+    torch.cuda.synchronize()
+    return {k: v.double().cpu().numpy() for k, v in g.items()}
+
+
+def check_grads(handle, inp, seed=3):
+    du, dl = _cotangents(inp, seed)
+    got = run_backward(handle, inp, du, dl)
+    ref = bw.ipa_vjp(inp, du, dl)
+    errs = {}
+    for key in bw.FLOAT_KEYS:
+        scale = float(np.max(np.abs(ref[key])))
+        err = float(np.max(np.abs(got[key] - ref[key])))
+        errs[key] = err / scale if scale > 0 else err
+    print({k: f"{v:.2e}" for k, v in errs.items()})
+    bad = {k: v for k, v in errs.items() if v > GRAD_TOL}
+    assert not bad, bad
+    # masked residues pass no gradient back
+    dead = ~np.asarray(inp["mask"]).astype(bool)
+    if dead.any():
+        for key in ("q", "k", "v", "q_points", "k_points", "v_points", "rotation", "translation", "z1", "z2"):
+            assert np.all(got[key][dead] == 0.0), key
+    return errs
+
+
+def _custom(seed, **kw):
+    base = dict(B=2, N=40, H=3, D=5, Dv=3, P=3, Q=5, Cz=7, R=3, Cout=20)
+    base.update(kw)
+    wl = workloads.Workload("edge", 9, dtype="bf16", frames="walk", t_scale=3.8, **base)
+    return workloads.make_inputs(wl, seed=seed)
+
+
+def test_backward_small_masks_and_empty_rows(handle):
+    inp = _custom(7, N=40)
+    rng = np.random.default_rng(7)
+    inp["mask"] = rng.random(inp["mask"].shape) < 0.8
+    inp["mask"][1, 30:] = False
+    pm = rng.random((2, 40, 40)) < 0.7
+    pm[0, 3, :] = False                                   # an empty neighbourhood
+    inp["pair_mask"] = pm
+    check_grads(handle, inp)
+
+
+@pytest.mark.parametrize("N", [1, 129, 300])
+def test_backward_ragged_tiles(handle, N):
+    inp = _custom(100 + N, N=N, B=1 if N == 300 else 2)
+    check_grads(handle, inp, seed=N)
+
+
+def test_backward_protein_batch(handle):
+    """Two samples of the protein-batch workload (B=8, N=256, Cz=128), padded
+    lengths masked."""
+    inp = workloads.make_inputs(workloads.workload(1).with_(B=2))
+    check_grads(handle, inp)
+
+
+def test_backward_long_chain_multi_tile(handle):
+    """Four query and key tiles of one chain (the length-sweep recipe, N=512)."""
+    check_grads(handle, workloads.make_inputs(workloads.workload("3-512")))
+
+
+def test_backward_rna_dims(handle):
+    """The RNA-chain widths (D=32, P=8, Cz=64) on a 256-residue chain."""
+    check_grads(handle, workloads.make_inputs(workloads.workload(2).with_(N=256)))
+
+
+def test_backward_short_chain_batch(handle):
+    """Four samples of the short-chain batch (N=150, lengths U{40..150})."""
+    inp = workloads.make_inputs(workloads.workload(4).with_(B=4))
+    check_grads(handle, inp)
+
+
+def test_backward_deterministic(handle):
+    inp = _custom(11, N=200)
+    du, dl = _cotangents(inp, 5)
+    a = run_backward(handle, inp, du, dl)
+    b = run_backward(handle, inp, du, dl)
+    for key in a:
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_backward_rejects_float32(handle):
+    from protein_structure_models_b200 import Fipa
+    from protein_structure_models_b200.fipa import FipaError
+    h = Fipa("f32", 0)
+    try:
+        inp = workloads.make_inputs(workloads.workload(0))
+        dev = to_device(inp, "f32")
+        du = torch.zeros((1, 32, 32), dtype=torch.float32, device="cuda")
+        with pytest.raises(FipaError, match="UNSUPPORTED"):
+            h.backward(dev, du, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
+    finally:
+        h.close()
