@@ -61,6 +61,8 @@ def parse_args():
                          "batch split across ranks (strong scaling); auto = rows for a single-sample "
                          "workload, replicas otherwise")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="leave the backward pass (training step) out of the bench line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--sweep", action="store_true",
                     help="length sweep N=512..32768 only: time, peak memory, fitted exponents (JSON lines)")
@@ -79,6 +81,16 @@ def flops_per_pair(wl) -> int:
     ka = wl.D + 3 * wl.P + wl.R * wl.Cz
     va = wl.Dv + 3 * wl.Q + wl.R * wl.Cz
     return 2 * ka + 2 * va
+
+
+def bwd_flops_per_pair(wl) -> int:
+    """Algorithmic flops of the backward's contractions per (b,h,i,j), counted
+    as flash-attention backward passes are: the logits once (2 Ka), dP (2 Va),
+    dQhat (2 Ka), dKhat (2 Ka), dVhat (2 Va) = 6 Ka + 4 Va.  The second
+    recompute of S and dP (one per side) is not counted."""
+    ka = wl.D + 3 * wl.P + wl.R * wl.Cz
+    va = wl.Dv + 3 * wl.Q + wl.R * wl.Cz
+    return 6 * ka + 4 * va
 
 
 def pair_counts(wl, inp):
@@ -163,6 +175,8 @@ KERNEL_SOURCES = {
     "fipa_lift_kernel": ("prologue.cu", "sm100.cuh", "plan.h", "kernels.h"),
     "fipa_core_kernel": ("core.cu", "sm100.cuh", "plan.h", "kernels.h"),
     "fipa_out_proj_kernel": ("epilogue.cu", "sm100.cuh", "plan.h", "kernels.h"),
+    "bwd_q_kernel": ("backward.cu", "sm100.cuh", "plan.h", "bwd_plan.h", "kernels.h"),
+    "bwd_k_kernel": ("backward.cu", "sm100.cuh", "plan.h", "bwd_plan.h", "kernels.h"),
 }
 
 
@@ -405,6 +419,67 @@ def run_fipa(args, wl, rank, world, local_rank):
     h.enable_stage_timing(False)
     core_ms = stage_sum["core"] / nb
 
+    # ---- backward (training step): fipa_backward replayed from a graph, L2
+    # flushed between steps; stage breakdown from a second graph with the
+    # library's events (not part of the timed steps)
+    bwd = None
+    if wl.dtype == "bf16" and mode == "replicas" and not args.no_backward:
+        from protein_structure_models_b200.fipa import Fipa as _F
+        rng = np.random.default_rng(wl.seed + 31)
+        d_update = torch.from_numpy(rng.standard_normal((wl.B, wl.N, wl.Cout)).astype(np.float32)).to(dev)
+        d_local = torch.from_numpy(rng.standard_normal((wl.B, wl.N, wl.H, wl.Q, 3)).astype(np.float32)).to(dev)
+        bws = torch.empty(h.backward_workspace_size(dims), dtype=torch.uint8, device=dev)
+        grads = {key: torch.empty(d_in[key].shape, dtype=torch.float32, device=dev) for key in _F.GRAD_KEYS.values()}
+
+        def backward(st):
+            h.backward(d_in, d_update, d_local, eps=inp["eps"], workspace=bws, grads=grads, stream=st)
+
+        backward(stream)
+        torch.cuda.synchronize()
+        h.sync_status()
+
+        def bcapture(stage_timing):
+            h.enable_stage_timing(stage_timing)
+            g = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cap):
+                backward(cap)
+            torch.cuda.synchronize()
+            return g
+
+        bgraph = bcapture(False)
+        sbgraph = bcapture(True)
+        nbs = max(3, min(args.steps, 20))
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            bgraph.replay()
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nbs)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for k in range(nbs):
+            flush.zero_()
+            bev[k][0].record(stream)
+            bgraph.replay()
+            bev[k][1].record(stream)
+        torch.cuda.synchronize()
+        h.sync_status()
+        bwd_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in bev) / nbs, dev)
+        bst = {}
+        for _ in range(nbs):
+            flush.zero_()
+            sbgraph.replay()
+            for name, ms in h.backward_stage_times().items():
+                bst[name] = bst.get(name, 0.0) + ms
+        torch.cuda.synchronize()
+        h.sync_status()
+        del bgraph, sbgraph
+        h.enable_stage_timing(False)
+        bwd = {"ms": bwd_ms, "steps": nbs, "stage_ms": {k: v / nbs for k, v in bst.items()},
+               "launches_per_call": 11}
+        del bws, grads
+
     # ---- end to end through the public API: each step copies its inputs from
     # pinned host memory (one packed buffer), runs the forward and copies the
     # update and local points back (one packed buffer).  Two steps are in
@@ -477,7 +552,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     h.close()
     return dict(inp=inp, mode=mode, step_ms=step_ms_max, core_ms=core_ms, launches=launches,
                 stage_ms={k: v / nb for k, v in stage_sum.items()}, clocks=clk,
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h)
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bwd=bwd)
 
 
 def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src, rows):
@@ -559,6 +634,22 @@ def main_fipa(args, wl):
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    if r["bwd"] is not None:
+        b = r["bwd"]
+        bf = bwd_flops_per_pair(wl)
+        gemm_ms = b["stage_ms"]["q_side"] + b["stage_ms"]["k_side"]
+        ach = bf * valid / (gemm_ms / 1e3) / 1e12
+        line["backward"] = {
+            "ms": b["ms"], "train_step_ms": r["step_ms"] + b["ms"],
+            "pairs_per_s": padded * mult / (b["ms"] / 1e3),
+            "train_step_pairs_per_s": padded * mult / ((r["step_ms"] + b["ms"]) / 1e3),
+            "stage_ms": b["stage_ms"], "steps": b["steps"],
+            "roofline": {"bound": "tensor", "kernel": "bwd_q_kernel + bwd_k_kernel", "achieved": ach,
+                         "peak": burst, "unit": "TFLOP/s", "frac": ach / burst,
+                         "work": f"{bf} flop per valid (b,h,i,j) (6 Ka + 4 Va) x {valid} valid pairs; "
+                                 f"time = q-side + k-side stages"},
+            "how": "fipa_backward (recomputes the lift and the core, then the backward kernels) replayed from "
+                   "a CUDA graph, L2 flushed between steps; cotangents N(0,1)"}
     if world == 1 and wl.index == 3 and not args.no_sweep:
         line["sweep"] = run_sweep(args.warmup)
     print(json.dumps(line), flush=True)

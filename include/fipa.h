@@ -265,6 +265,15 @@ fipa_status fipa_backward(fipa_handle* h,
                           void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Device time in milliseconds of each stage of the most recent fipa_backward
+ * recorded with stage timing on (fipa_enable_stage_timing), in launch order:
+ * [0] recompute (lift and fused core), [1] cotangent preparation (d_update @
+ * w_out^T and the per-residue dO rows), [2] q-side kernel (dS, dQhat), [3]
+ * k-side kernel (dKhat, dVhat, dz2), [4] chain rule through frames and
+ * factors and the weight gradients.  Waits for that call's last event. */
+#define FIPA_BWD_STAGES 5
+fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n);
+
 /* Wait for `stream`, then read and clear the handle's device status word.
  * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */
@@ -282,6 +291,7 @@ fipa_status fipa_selftest_timeout(fipa_handle* h, unsigned timeout_ms, void* str
  * calls on this handle record a CUDA event before and after each of their
  * kernels on the call's stream; the events are created here, so fipa_forward
  * still allocates nothing.  `enable` = 0 turns recording off and frees them.
+ * fipa_backward calls record their own stage events the same way.
  * A CUDA graph captured from a timed call records into these events on every
  * replay: release such a graph before turning timing off. */
 fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable);

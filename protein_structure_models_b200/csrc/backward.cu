@@ -1452,7 +1452,11 @@ size_t bwd_chain_smem(const Plan& p) {
 
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s) {
+                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s,
+                            StageMark mark, void* mark_ctx) {
+  auto stage = [&](int k) {
+    if (mark != nullptr) mark(mark_ctx, k);
+  };
   BwdArgs a;
   a.p = p;
   a.bp = bp;
@@ -1481,6 +1485,7 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   a.timeout_ns = ctl.timeout_ns;
   const int BN = p.B * p.N;
   cudaError_t e;
+  stage(1);
   bwd_dfeat_kernel<<<dim3(cdiv(p.F, 64), cdiv(BN, 64)), 256, 0, s>>>(
       io.d_update, static_cast<const __nv_bfloat16*>(in.w_out), a.dfeat, BN, p.F, p.Cout);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1492,11 +1497,14 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   bwd_prep_kernel<<<BN, 256, psm, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_q_kernel))) != cudaSuccess) return e;
+  stage(2);
   bwd_q_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.q_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_k_kernel))) != cudaSuccess) return e;
+  stage(3);
   bwd_k_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.k_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stage(4);
   const size_t csm = bwd_chain_smem(p);
   if (csm > 48 * 1024) {
     if ((e = cudaFuncSetAttribute(bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csm)) != cudaSuccess)
@@ -1512,7 +1520,9 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
                                                                       p.Cout, bp.dw_ks);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   bwd_final_kernel<<<cdiv(p.Cz * p.H + p.H, 256), 256, 0, s>>>(a);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  stage(5);
+  return cudaSuccess;
 }
 
 }  // namespace fipa

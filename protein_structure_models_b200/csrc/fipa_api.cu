@@ -21,6 +21,8 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 // stage-timing intervals: prologue, core, output projection, attention output
 constexpr int kStages = FIPA_STAGES;
+// backward: recompute, prep, q side, k side, chain and weight gradients
+constexpr int kBwdStages = FIPA_BWD_STAGES;
 
 struct fipa_handle {
   int device = 0;
@@ -34,6 +36,8 @@ struct fipa_handle {
   bool timing = false;
   bool timed_call = false;
   cudaEvent_t ev[kStages + 1] = {};
+  cudaEvent_t bev[kBwdStages + 1] = {};   // backward stage events (with stage timing on)
+  bool bwd_timed_call = false;
   long long* d_trace = nullptr;
   int trace_cta = -1;
   int pair_split = 1;
@@ -231,12 +235,18 @@ FIPA_API fipa_status fipa_enable_stage_timing(fipa_handle* h, int enable) {
       cudaError_t err = cudaEventCreate(&e);
       if (err != cudaSuccess) return cuda_fail(h, "event create", err);
     }
+    for (auto& e : h->bev) {
+      cudaError_t err = cudaEventCreate(&e);
+      if (err != cudaSuccess) return cuda_fail(h, "event create", err);
+    }
     h->timing = true;
   } else if (!enable && h->timing) {
     for (auto& e : h->ev) { cudaEventDestroy(e); e = nullptr; }
+    for (auto& e : h->bev) { cudaEventDestroy(e); e = nullptr; }
     h->timing = false;
   }
   h->timed_call = false;
+  h->bwd_timed_call = false;
   return FIPA_OK;
 }
 
@@ -261,8 +271,10 @@ FIPA_API fipa_status fipa_destroy(fipa_handle* h) {
     DeviceGuard g(h->device);
     if (h->d_status) cudaFree(h->d_status);
     if (h->d_trace) cudaFree(h->d_trace);
-    if (h->timing)
+    if (h->timing) {
       for (auto& e : h->ev) cudaEventDestroy(e);
+      for (auto& e : h->bev) cudaEventDestroy(e);
+    }
   }
   delete h;
   return FIPA_OK;
@@ -550,11 +562,44 @@ FIPA_API fipa_status fipa_backward(fipa_handle* h, const void* q, const void* k,
                                 grads->b_out},
                  ws};
   cudaError_t e;
+  struct Marker {
+    fipa_handle* h;
+    cudaStream_t s;
+    unsigned flags;
+  } mk{h, s, cudaEventRecordDefault};
+  const bool rec = h->timing;
+  if (rec) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cap);
+    mk.flags = cap == cudaStreamCaptureStatusActive ? cudaEventRecordExternal : cudaEventRecordDefault;
+  }
+  auto mark = [](void* ctx, int k) {
+    Marker* m = static_cast<Marker*>(ctx);
+    cudaEventRecordWithFlags(m->h->bev[k], m->s, m->flags);
+  };
+  if (rec) mark(&mk, 0);
   // recompute: the lift, and the core saving the normalised aggregates
   if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
   if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
     return cuda_fail(h, "core launch", e);
-  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, ctl, s)) != cudaSuccess)
+  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, ctl, s,
+                                 rec ? +mark : nullptr, &mk)) != cudaSuccess)
     return cuda_fail(h, "backward launch", e);
+  h->bwd_timed_call = rec;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n) {
+  if (h == nullptr || ms == nullptr || n < 0) return FIPA_ERR_INVALID_ARG;
+  if (!h->timing || !h->bwd_timed_call) return fail(h, FIPA_ERR_INVALID_ARG, "no timed fipa_backward call");
+  DeviceGuard g(h->device);
+  cudaError_t e = cudaEventSynchronize(h->bev[kBwdStages]);
+  if (e != cudaSuccess) return cuda_fail(h, "event sync", e);
+  for (int k = 0; k < kBwdStages && k < n; ++k) {
+    float t = 0.f;
+    e = cudaEventElapsedTime(&t, h->bev[k], h->bev[k + 1]);
+    if (e != cudaSuccess) return cuda_fail(h, "event time", e);
+    ms[k] = t;
+  }
   return FIPA_OK;
 }

@@ -112,9 +112,13 @@ struct BwdIO {
 };
 // The backward kernels after the recompute (lift, and the core with the
 // aggregates saved at the BwdPlan's osave offset).
+// `mark(ctx, k)`, if given, is called before stage k = 1 (dfeat GEMM and prep),
+// 2 (q side), 3 (k side), 4 (chain and weight gradients) and after the last (5).
+typedef void (*StageMark)(void* ctx, int k);
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s);
+                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s,
+                            StageMark mark = nullptr, void* mark_ctx = nullptr);
 
 // Per-head distance weight 1/2 softplus(raw) sqrt(2/(27P)), softplus without overflow.
 __device__ __forceinline__ float point_weight(float raw, int P) {

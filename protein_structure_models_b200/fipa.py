@@ -95,6 +95,8 @@ def load_library():
     lib.fipa_backward.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double, ctypes.POINTER(FipaDims)] \
         + [vp, vp, ctypes.POINTER(FipaGrads), vp, sz, vp]
     lib.fipa_backward.restype = c_int
+    lib.fipa_backward_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), c_int]
+    lib.fipa_backward_stage_times.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -259,6 +261,14 @@ class Fipa:
                                     ctypes.c_void_p(s.cuda_stream))
         self._check(st)
         return grads
+
+    BWD_STAGES = ("recompute", "prep", "q_side", "k_side", "chain")
+
+    def backward_stage_times(self) -> dict:
+        """Device ms of each stage of the most recent timed backward."""
+        buf = (ctypes.c_float * len(self.BWD_STAGES))()
+        self._check(self.lib.fipa_backward_stage_times(self.handle, buf, len(self.BWD_STAGES)))
+        return dict(zip(self.BWD_STAGES, [float(x) for x in buf]))
 
     STAGES = ("prologue", "core", "out_proj", "attention")
 

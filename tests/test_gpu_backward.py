@@ -136,3 +136,17 @@ def test_backward_rejects_float32(handle):
             h.backward(dev, du, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
     finally:
         h.close()
+
+
+def test_backward_stage_times(handle):
+    """With stage timing on, fipa_backward records its five stages."""
+    inp = _custom(13, N=129)
+    du, dl = _cotangents(inp, 2)
+    handle.enable_stage_timing(True)
+    try:
+        run_backward(handle, inp, du, dl)
+        st = handle.backward_stage_times()
+    finally:
+        handle.enable_stage_timing(False)
+    assert list(st) == ["recompute", "prep", "q_side", "k_side", "chain"]
+    assert all(v > 0.0 for v in st.values()), st
