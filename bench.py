@@ -61,6 +61,7 @@ def parse_args():
                          "batch split across ranks (strong scaling); auto = rows for a single-sample "
                          "workload, replicas otherwise")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-knn", action="store_true", help="leave the kNN distogram timing out of the bench line")
     ap.add_argument("--no-backward", action="store_true",
                     help="leave the backward pass (training step) out of the bench line")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -480,6 +481,35 @@ def run_fipa(args, wl, rank, world, local_rank):
                "launches_per_call": 11}
         del bws, grads
 
+    # ---- kNN distogram features of the same structures (k = 20, 39 bins)
+    knn = None
+    if not args.no_knn:
+        from protein_structure_models_b200.fipa import knn_distogram
+        kk, nb = 20, 39
+        edges = torch.linspace(3.25, 50.75, nb - 1, device=dev, dtype=torch.float32)
+        kout = {"idx": torch.empty((wl.B, wl.N, kk), dtype=torch.int32, device=dev),
+                "dist": torch.empty((wl.B, wl.N, kk), dtype=torch.float32, device=dev),
+                "bin": torch.empty((wl.B, wl.N, kk), dtype=torch.int32, device=dev),
+                "onehot": torch.empty((wl.B, wl.N, kk, nb), dtype=torch.float32, device=dev)}
+        tr, mk = d_in["translation"], d_in["mask"]
+        for _ in range(3):
+            knn_distogram(tr, mk, kk, edges, out=kout, stream=stream)
+        torch.cuda.synchronize()
+        nk = max(3, min(args.steps, 50))
+        kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nk)]
+        for k in range(nk):
+            flush.zero_()
+            kev[k][0].record(stream)
+            knn_distogram(tr, mk, kk, edges, out=kout, stream=stream)
+            kev[k][1].record(stream)
+        torch.cuda.synchronize()
+        knn_ms = sum(a.elapsed_time(b) for a, b in kev) / nk
+        knn = {"ms": knn_ms, "k": kk, "n_bins": nb, "steps": nk,
+               "pairs_per_s": wl.B * wl.N * wl.N / (knn_ms / 1e3),
+               "how": "fipa_knn_distogram on the workload's translations and mask (indices, distances, bins, "
+                      "one-hot [B,N,k,n_bins]); every query scans all keys of its sample, block-wise"}
+        del kout
+
     # ---- end to end through the public API: each step copies its inputs from
     # pinned host memory (one packed buffer), runs the forward and copies the
     # update and local points back (one packed buffer).  Two steps are in
@@ -552,7 +582,7 @@ def run_fipa(args, wl, rank, world, local_rank):
     h.close()
     return dict(inp=inp, mode=mode, step_ms=step_ms_max, core_ms=core_ms, launches=launches,
                 stage_ms={k: v / nb for k, v in stage_sum.items()}, clocks=clk,
-                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bwd=bwd)
+                e2e_ms=e2e_ms, h2d=h2d, d2h=d2h, bwd=bwd, knn=knn)
 
 
 def kernel_rooflines(wl, stage_ms, valid, fpp, burst, hbm, src, rows):
@@ -650,6 +680,8 @@ def main_fipa(args, wl):
                                  f"time = q-side + k-side stages"},
             "how": "fipa_backward (recomputes the lift and the core, then the backward kernels) replayed from "
                    "a CUDA graph, L2 flushed between steps; cotangents N(0,1)"}
+    if r["knn"] is not None:
+        line["knn_distogram"] = r["knn"]
     if world == 1 and wl.index == 3 and not args.no_sweep:
         line["sweep"] = run_sweep(args.warmup)
     print(json.dumps(line), flush=True)

@@ -274,6 +274,33 @@ fipa_status fipa_backward(fipa_handle* h,
 #define FIPA_BWD_STAGES 5
 fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n);
 
+/* k-nearest-neighbour distogram features ("Flash Invariant Point Attention",
+ * rebuttal answer 6: keep the k nearest neighbours of each residue,
+ * (B, L, k, n_bins), instead of the (B, L, L, n_bins) distogram; found
+ * block-wise, without an L x L matrix).
+ *   trans       [B,N,3]  frame translations (float32 or bfloat16 as `dtype`)
+ *   mask        [B,N]    uint8, 1 = valid residue
+ *   k           1..32 neighbours per residue (the pages use 20)
+ *   edges       [n_bins - 1] float32, ascending; the bin of a distance d is the
+ *               number of edges e <= d (NULL allowed when n_bins == 1)
+ * Outputs (device, caller-owned):
+ *   out_idx     [B,N,k] int32   neighbour residue indices, nearest first; the
+ *               neighbours of i are the valid residues of its sample, i itself
+ *               included; ties in distance go to the smaller index
+ *   out_dist    [B,N,k] float32 distances (+inf for an empty slot)
+ *   out_bin     [B,N,k] int32   distogram bins (-1 for an empty slot)
+ *   out_onehot  [B,N,k,n_bins] float32 one-hot bins, or NULL
+ * A masked residue has no neighbours (all slots empty); a sample with fewer
+ * than k valid residues leaves the remaining slots empty.  The order is decided
+ * on the squared distance ((dx dx) + (dy dy)) + (dz dz), each operation rounded
+ * to float32.  No handle: every pointer belongs to the current device.
+ * Allocates nothing; runs on `stream`.  FIPA_ERR_UNSUPPORTED for k > 32 or
+ * B > 65535. */
+fipa_status fipa_knn_distogram(fipa_dtype dtype, const void* trans, const uint8_t* mask,
+                               int B, int N, int k, const float* edges, int n_bins,
+                               int32_t* out_idx, float* out_dist, int32_t* out_bin,
+                               float* out_onehot, void* stream);
+
 /* Wait for `stream`, then read and clear the handle's device status word.
  * Returns FIPA_ERR_DEVICE_TIMEOUT if a kernel gave up on a bounded wait since
  * the last call, FIPA_ERR_CUDA if the stream reports an error, else FIPA_OK. */

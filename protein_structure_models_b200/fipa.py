@@ -97,6 +97,8 @@ def load_library():
     lib.fipa_backward.restype = c_int
     lib.fipa_backward_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), c_int]
     lib.fipa_backward_stage_times.restype = c_int
+    lib.fipa_knn_distogram.argtypes = [c_int, vp, vp, c_int, c_int, c_int, vp, c_int, vp, vp, vp, vp, vp]
+    lib.fipa_knn_distogram.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -324,6 +326,41 @@ def forward_noalloc(inp: dict, eps: float = 1e-8, out: Optional[dict] = None,
             ctypes.c_void_p(s.cuda_stream))
     if st != FIPA_OK:
         raise FipaError(st, "fipa_forward_noalloc failed")
+    return out
+
+
+def knn_distogram(translation: torch.Tensor, mask: torch.Tensor, k: int, edges: torch.Tensor,
+                  onehot: bool = True, out: Optional[dict] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """fipa_knn_distogram: the k nearest valid residues of every residue (self
+    included, ties to the smaller index) and their distogram bins.
+    translation [B,N,3] float32/bfloat16, mask [B,N] bool/uint8, edges
+    [n_bins - 1] float32 ascending, all on one CUDA device.  Returns idx [B,N,k]
+    int32, dist [B,N,k] float32, bin [B,N,k] int32 and (with onehot)
+    onehot [B,N,k,n_bins] float32."""
+    lib = load_library()
+    dev = translation.device
+    B, N, _ = translation.shape
+    n_bins = edges.numel() + 1
+    for name, t in (("translation", translation), ("mask", mask), ("edges", edges)):
+        if t.device != dev or not t.is_contiguous():
+            raise ValueError(f"{name}: need a contiguous tensor on {dev}")
+    if translation.dtype not in (torch.float32, torch.bfloat16) or edges.dtype != torch.float32:
+        raise ValueError("translation must be float32 or bfloat16, edges float32")
+    with torch.cuda.device(dev):
+        if out is None:
+            out = {"idx": torch.empty((B, N, k), dtype=torch.int32, device=dev),
+                   "dist": torch.empty((B, N, k), dtype=torch.float32, device=dev),
+                   "bin": torch.empty((B, N, k), dtype=torch.int32, device=dev)}
+            if onehot:
+                out["onehot"] = torch.empty((B, N, k, n_bins), dtype=torch.float32, device=dev)
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        st = lib.fipa_knn_distogram(F32 if translation.dtype == torch.float32 else BF16, _ptr(translation),
+                                    _ptr(mask), B, N, k, _ptr(edges) if edges.numel() else None, n_bins,
+                                    _ptr(out["idx"]), _ptr(out["dist"]), _ptr(out["bin"]), _ptr(out.get("onehot")),
+                                    ctypes.c_void_p(s.cuda_stream))
+    if st != FIPA_OK:
+        raise FipaError(st, "fipa_knn_distogram failed")
     return out
 
 
