@@ -274,6 +274,34 @@ fipa_status fipa_backward(fipa_handle* h,
 #define FIPA_BWD_STAGES 5
 fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n);
 
+/* The IPA layer around the core (float32 handle).  The page "Invariant point
+ * attention (IPA)" (Required behavior) defines the core as starting after the
+ * input projections and ending before any residual or frame update, and asks
+ * not to invent weights; this layer applies the plainest forms of those steps
+ * with every weight supplied by the caller:
+ *   X = s @ W_in + b_in                      s [B,N,Cs], W_in [Cs,Din], b_in [Din]
+ *       split in order into q [H,D], k [H,D], v [H,Dv], q_pts [H,P,3],
+ *       k_pts [H,P,3], v_pts [H,Q,3], z1 [R,Cz], z2 [R,Cz] (row-major blocks),
+ *       Din = H(2D + Dv) + 3H(2P + Q) + 2 R Cz
+ *   the fused core with rot, trans, masks, Wb, point_w_raw, w_out [F,Cs], b_out [Cs]
+ *   s' = s + update                          -> out_s [B,N,Cs]
+ *   [b c d tx ty tz] = s' @ W_bb + b_bb      W_bb [Cs,6], b_bb [6]
+ *   R' = R R(q), q = (1,b,c,d)/|(1,b,c,d)|;  t' = R (tx,ty,tz) + t
+ *                                            -> out_rot [B,N,3,3], out_trans [B,N,3]
+ *   (a masked residue keeps its frame), and the core's local points.
+ * dims->Cout must equal Cs.  All pointers float32 device buffers except the
+ * masks; workspace >= fipa_layer_workspace_size() bytes, 256-byte aligned.
+ * FIPA_ERR_UNSUPPORTED with a bfloat16 handle.  Allocates nothing; runs on
+ * `stream`. */
+fipa_status fipa_layer_workspace_size(const fipa_handle* h, const fipa_dims* dims, size_t* bytes);
+fipa_status fipa_ipa_layer(fipa_handle* h, const float* s, const float* W_in, const float* b_in,
+                           const float* rot, const float* trans, const uint8_t* mask,
+                           const uint8_t* pair_mask, const float* Wb, const float* point_w_raw,
+                           const float* w_out, const float* b_out, const float* W_bb,
+                           const float* b_bb, double eps, const fipa_dims* dims,
+                           float* out_s, float* out_rot, float* out_trans, float* out_local_points,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
 /* k-nearest-neighbour distogram features ("Flash Invariant Point Attention",
  * rebuttal answer 6: keep the k nearest neighbours of each residue,
  * (B, L, k, n_bins), instead of the (B, L, L, n_bins) distogram; found

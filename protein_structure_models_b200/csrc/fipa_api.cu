@@ -603,3 +603,90 @@ FIPA_API fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n)
   }
   return FIPA_OK;
 }
+
+// ---------------------------------------------------------------- IPA layer
+namespace {
+struct LayerLayout {
+  int Din;
+  int start[9];
+  size_t off_blk[8], off_upd, total;
+};
+
+void layer_layout(const Plan& p, LayerLayout& L) {
+  const int widths[8] = {p.H * p.D, p.H * p.D, p.H * p.Dv, p.H * p.P * 3, p.H * p.P * 3, p.H * p.Q * 3,
+                         p.R * p.Cz, p.R * p.Cz};
+  const size_t BN = (size_t)p.B * p.N;
+  L.start[0] = 0;
+  size_t o = fipa::rup_sz(p.total, 256);
+  for (int i = 0; i < 8; ++i) {
+    L.start[i + 1] = L.start[i] + widths[i];
+    L.off_blk[i] = o;
+    o = fipa::rup_sz(o + BN * widths[i] * 4, 256);
+  }
+  L.Din = L.start[8];
+  L.off_upd = o;
+  o = fipa::rup_sz(o + BN * p.Cout * 4, 256);
+  L.total = o;
+}
+}  // namespace
+
+FIPA_API fipa_status fipa_layer_workspace_size(const fipa_handle* hc, const fipa_dims* dims, size_t* bytes) {
+  fipa_handle* h = const_cast<fipa_handle*>(hc);
+  if (h == nullptr || dims == nullptr || bytes == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "null argument");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  LayerLayout L;
+  layer_layout(p, L);
+  *bytes = L.total;
+  return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_ipa_layer(fipa_handle* h, const float* s, const float* W_in, const float* b_in,
+                                    const float* rot, const float* trans, const uint8_t* mask,
+                                    const uint8_t* pair_mask, const float* Wb, const float* point_w_raw,
+                                    const float* w_out, const float* b_out, const float* W_bb, const float* b_bb,
+                                    double eps, const fipa_dims* dims, float* out_s, float* out_rot,
+                                    float* out_trans, float* out_local_points, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
+  if (h->dtype != FIPA_F32) return fail(h, FIPA_ERR_UNSUPPORTED, "the IPA layer runs with a float32 handle");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  const void* req[] = {s, W_in, b_in, rot, trans, mask, Wb, point_w_raw, w_out, b_out, W_bb, b_bb,
+                       out_s, out_rot, out_trans, out_local_points};
+  for (const void* ptr : req)
+    if (ptr == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "a required pointer is NULL");
+  const void* al[] = {s, W_in, b_in, rot, trans, Wb, point_w_raw, w_out, b_out, W_bb, b_bb, out_s, out_rot,
+                      out_trans, out_local_points};
+  for (const void* ptr : al)
+    if (!aligned(ptr, 4)) return fail(h, FIPA_ERR_INVALID_ARG, "a float pointer is misaligned");
+  LayerLayout L;
+  layer_layout(p, L);
+  if (workspace == nullptr || workspace_bytes < L.total)
+    return fail(h, FIPA_ERR_WORKSPACE, "layer workspace needs " + std::to_string(L.total) + " bytes");
+  if (!aligned(workspace, 256)) return fail(h, FIPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  DeviceGuard g(h->device);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* blk[8];
+  for (int i = 0; i < 8; ++i) blk[i] = reinterpret_cast<float*>(ws + L.off_blk[i]);
+  float* upd = reinterpret_cast<float*>(ws + L.off_upd);
+  const int M = p.B * p.N;
+  cudaError_t e;
+  if ((e = fipa::launch_layer_proj(s, W_in, b_in, M, p.Cout, L.Din, blk, L.start, st)) != cudaSuccess)
+    return cuda_fail(h, "layer projection launch", e);
+  fipa_status fs = forward_impl(h, blk[0], blk[1], blk[2], blk[3], blk[4], blk[5], rot, trans, blk[6], blk[7], Wb,
+                                point_w_raw, mask, pair_mask, w_out, b_out, eps, dims, 0, -1, upd, out_local_points,
+                                nullptr, nullptr, workspace, p.total, stream);
+  if (fs != FIPA_OK) return fs;
+  if ((e = fipa::launch_layer_frame(s, upd, W_bb, b_bb, rot, trans, mask, M, p.Cout, out_s, out_rot, out_trans,
+                                    st)) != cudaSuccess)
+    return cuda_fail(h, "layer frame-update launch", e);
+  return FIPA_OK;
+}

@@ -120,6 +120,13 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
                             const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s,
                             StageMark mark = nullptr, void* mark_ctx = nullptr);
 
+// The IPA layer around the core (layer.cu), float32.
+cudaError_t launch_layer_proj(const float* s, const float* W_in, const float* b_in, int M, int Cs, int Din,
+                              float* const dst[8], const int start[9], cudaStream_t st);
+cudaError_t launch_layer_frame(const float* s, const float* upd, const float* W_bb, const float* b_bb, const float* rot,
+                               const float* trans, const uint8_t* mask, int M, int Cs, float* out_s, float* out_rot,
+                               float* out_trans, cudaStream_t st);
+
 // Per-head distance weight 1/2 softplus(raw) sqrt(2/(27P)), softplus without overflow.
 __device__ __forceinline__ float point_weight(float raw, int P) {
   const float sp = raw > 0.f ? raw + log1pf(expf(-raw)) : log1pf(expf(raw));

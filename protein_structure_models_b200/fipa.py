@@ -99,6 +99,11 @@ def load_library():
     lib.fipa_backward_stage_times.restype = c_int
     lib.fipa_knn_distogram.argtypes = [c_int, vp, vp, c_int, c_int, c_int, vp, c_int, vp, vp, vp, vp, vp]
     lib.fipa_knn_distogram.restype = c_int
+    lib.fipa_layer_workspace_size.argtypes = [vp, ctypes.POINTER(FipaDims), ctypes.POINTER(sz)]
+    lib.fipa_layer_workspace_size.restype = c_int
+    lib.fipa_ipa_layer.argtypes = [vp] + [vp] * 5 + [vp, vp] + [vp] * 6 + [ctypes.c_double, ctypes.POINTER(FipaDims)] \
+        + [vp] * 4 + [vp, sz, vp]
+    lib.fipa_ipa_layer.restype = c_int
     lib.fipa_destroy.argtypes = [vp]
     lib.fipa_destroy.restype = c_int
     _lib = lib
@@ -263,6 +268,40 @@ class Fipa:
                                     ctypes.c_void_p(s.cuda_stream))
         self._check(st)
         return grads
+
+    def ipa_layer(self, inp: dict, dims: dict, eps: float = 1e-8, workspace: Optional[torch.Tensor] = None,
+                  stream: Optional[torch.cuda.Stream] = None) -> dict:
+        """fipa_ipa_layer (float32 handle): the projection, the core, the residual and
+        the frame update.  inp: s, W_in, b_in, rotation, translation, mask, pair_mask,
+        Wb, point_weight_raw, w_out, b_out, W_bb, b_bb (float32 CUDA tensors, masks
+        bool/uint8); dims: H, D, Dv, P, Q, Cz, R.  Returns s, rotation, translation,
+        local_points."""
+        dev = torch.device("cuda", self.device)
+        s = inp["s"]
+        B, N, Cs = s.shape
+        full = dict(B=B, N=N, Cout=Cs, **{k: dims[k] for k in ("H", "D", "Dv", "P", "Q", "Cz", "R")})
+        for k in ("s", "W_in", "b_in", "rotation", "translation", "Wb", "point_weight_raw", "w_out", "b_out",
+                  "W_bb", "b_bb"):
+            t = inp[k]
+            if t.dtype != torch.float32 or t.device != dev or not t.is_contiguous():
+                raise ValueError(f"{k}: need a contiguous float32 tensor on {dev}")
+        d = make_dims(**full)
+        if workspace is None:
+            n = ctypes.c_size_t()
+            self._check(self.lib.fipa_layer_workspace_size(self.handle, ctypes.byref(d), ctypes.byref(n)))
+            workspace = torch.empty(int(n.value), dtype=torch.uint8, device=dev)
+        out = {"s": torch.empty_like(s), "rotation": torch.empty_like(inp["rotation"]),
+               "translation": torch.empty_like(inp["translation"]),
+               "local_points": torch.empty((B, N, dims["H"], dims["Q"], 3), dtype=torch.float32, device=dev)}
+        st = stream if stream is not None else torch.cuda.current_stream(dev)
+        self._check(self.lib.fipa_ipa_layer(
+            self.handle, _ptr(s), _ptr(inp["W_in"]), _ptr(inp["b_in"]), _ptr(inp["rotation"]),
+            _ptr(inp["translation"]), _ptr(inp["mask"]), _ptr(inp.get("pair_mask")), _ptr(inp["Wb"]),
+            _ptr(inp["point_weight_raw"]), _ptr(inp["w_out"]), _ptr(inp["b_out"]), _ptr(inp["W_bb"]),
+            _ptr(inp["b_bb"]), float(eps), ctypes.byref(d), _ptr(out["s"]), _ptr(out["rotation"]),
+            _ptr(out["translation"]), _ptr(out["local_points"]), _ptr(workspace),
+            ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(st.cuda_stream)))
+        return out
 
     BWD_STAGES = ("recompute", "prep", "q_side", "k_side", "chain")
 
