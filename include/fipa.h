@@ -89,6 +89,8 @@ typedef struct fipa_handle fipa_handle;
  *                              query tile then stream with the keys); 1 (default)
  *                              from 8 key tiles per sample up, 2 wherever it
  *                              fits, 0 never
+ *   FIPA_RING_STAGES=2..8      tuning: cap the shared-memory ring stages of the
+ *                              core and backward kernels (default: as many as fit)
  *   FIPA_TRACE_CTA=<n>         debug trace of one core CTA (see fipa_trace_copy) */
 fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims,
                         fipa_dtype dtype, int device);

@@ -492,7 +492,6 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       tc_fence_after();
       Ring rg{full, empty, sRing, bp.q_nst};
       const uint32_t idS = idesc_f16(128, 128, 0, 0);
-      const uint32_t idQ = idesc_f16(128, 64, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sOa = smem_u32(sO);
       auto take = [&](int site) -> int {
         if (!mbar_wait(&full[rg.st], rg.ph, wc, site)) return -1;
@@ -547,17 +546,28 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tc_commit(dp_full);
         return true;
       };
+      // dQhat += dS [KH | Z]: chunks in consecutive ring slots form one MMA of
+      // N = 64 x run (up to 4), into consecutive 64-column blocks of dQhat
       auto mma_dq = [&](int s) -> bool {
-        for (int c = 0; c < nKH + nZ; ++c) {
-          const int sk = take(25);
-          if (sk < 0) return false;
-          const uint32_t bk = ringa + sk * kChunkBytes;
+        const int nch = nKH + nZ;
+        for (int c = 0; c < nch;) {
+          int run = nch - c;
+          if (run > 4) run = 4;
+          if (run > rg.nst - rg.st) run = rg.nst - rg.st;
+          for (int u = 0; u < run; ++u)
+            if (!mbar_wait(&full[rg.st + u], rg.ph, wc, 25)) return false;
+          tc_fence_after();
+          const uint32_t bk = ringa + rg.st * kChunkBytes;
           const uint32_t dcol = tmem + (uint32_t)(bp.tmDQ + c * kChunk);
+          const uint32_t idR = idesc_f16(128, 64 * run, 0, 1);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(dcol, tmem + (uint32_t)bp.tmDS + kk * 8, desc_mnmajor_sw128(bk + kk * 2048, kChunkBytes), idQ,
+            mma_ts(dcol, tmem + (uint32_t)bp.tmDS + kk * 8, desc_mnmajor_sw128(bk + kk * 2048, kChunkBytes), idR,
                    (s > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(&empty[sk]);
+          for (int u = 0; u < run; ++u) tc_commit(&empty[rg.st + u]);
+          rg.st += run;
+          if (rg.st == rg.nst) { rg.st = 0; rg.ph ^= 1u; }
+          c += run;
         }
         tc_commit(dq_done);
         return true;
@@ -917,13 +927,15 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       auto push_dp = [&](int qt) {
         for (int c = 0; c < bp.nOc; ++c) push(&tmdO, c * kChunk, qt);
       };
+      // gradient products: QH, dO head, then the u hi and dU chunks each as one
+      // run of consecutive ring slots (the dz2 product uses u hi only: the lo
+      // half is 2^-12 of u, far below the gradient tolerance; the logits above
+      // are recomputed with both halves)
       auto push_gr = [&](int qt) {
         for (int c = 0; c < nKH; ++c) push(&tmQ, c * kChunk, qt);
         for (int c = 0; c < nVH; ++c) push(&tmdO, c * kChunk, qt);
-        for (int c = 0; c < nZ; ++c) {
-          for (int qz = 0; qz < nqz; ++qz) push(&tmQ, (nKH + qz * nZ + c) * kChunk, qt);
-          push(&tmdO, (nVH + c) * kChunk, qt);
-        }
+        for (int c = 0; c < nZ; ++c) push(&tmQ, (nKH + c) * kChunk, qt);
+        for (int c = 0; c < nZ; ++c) push(&tmdO, (nVH + c) * kChunk, qt);
       };
       push_st(tiles[0]);
       push_dp(tiles[0]);
@@ -948,7 +960,6 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       tc_fence_after();
       Ring rg{full, empty, sRing, bp.k_nst};
       const uint32_t idS = idesc_f16(128, 128, 0, 0);
-      const uint32_t idG = idesc_f16(128, 64, 0, 1);
       const uint32_t sKa = smem_u32(sK), sPa = smem_u32(sP), sDa = smem_u32(sD), ringa = smem_u32(sRing);
       auto take = [&](int site) -> int {
         if (!mbar_wait(&full[rg.st], rg.ph, wc, site)) return -1;
@@ -1005,29 +1016,36 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         tc_commit(dp_full);
         return true;
       };
-      auto gr_one = [&](uint32_t dcol, uint32_t abase, bool acc0, int site) -> bool {
-        const int sl = take(site);
-        if (sl < 0) return false;
-        const uint32_t bq = ringa + sl * kChunkBytes;
+      // `nch` chunks into consecutive 64-column blocks from `dcol`: chunks in
+      // consecutive ring slots form one MMA of N = 64 x run (MN-major B, groups
+      // one slot apart), up to 4 chunks
+      auto gr_run = [&](uint32_t dcol, uint32_t abase, int nch, bool acc0, int site) -> bool {
+        for (int c = 0; c < nch;) {
+          int run = nch - c;
+          if (run > 4) run = 4;
+          if (run > rg.nst - rg.st) run = rg.nst - rg.st;
+          for (int u = 0; u < run; ++u)
+            if (!mbar_wait(&full[rg.st + u], rg.ph, wc, site)) return false;
+          tc_fence_after();
+          const uint32_t bq = ringa + rg.st * kChunkBytes;
+          const uint32_t idR = idesc_f16(128, 64 * run, 0, 1);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(dcol, adesc(abase, kk), desc_mnmajor_sw128(bq + kk * 2048, kChunkBytes), idG,
-                 (acc0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[sl]);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(dcol + (uint32_t)(c * kChunk), adesc(abase, kk), desc_mnmajor_sw128(bq + kk * 2048, kChunkBytes),
+                   idR, (acc0 || kk > 0) ? 1u : 0u);
+          for (int u = 0; u < run; ++u) tc_commit(&empty[rg.st + u]);
+          rg.st += run;
+          if (rg.st == rg.nst) { rg.st = 0; rg.ph ^= 1u; }
+          c += run;
+        }
         return true;
       };
       auto mma_gr = [&](int s) -> bool {
         const bool acc0 = s > 0;
-        for (int c = 0; c < nKH; ++c)
-          if (!gr_one(tmem + (uint32_t)(bp.tmDK + c * kChunk), sDa, acc0, 45)) return false;
-        for (int c = 0; c < nVH; ++c)
-          if (!gr_one(tmem + (uint32_t)(bp.tmDV + c * kChunk), sPa, acc0, 46)) return false;
-        for (int c = 0; c < nZ; ++c) {
-          const uint32_t dz = tmem + (uint32_t)(bp.tmDZ + c * kChunk);
-          for (int qz = 0; qz < nqz; ++qz)
-            if (!gr_one(dz, sDa, acc0 || qz > 0, 47)) return false;
-          if (!gr_one(dz, sPa, true, 48)) return false;
-        }
+        if (!gr_run(tmem + (uint32_t)bp.tmDK, sDa, nKH, acc0, 45)) return false;
+        if (!gr_run(tmem + (uint32_t)bp.tmDV, sPa, nVH, acc0, 46)) return false;
+        if (!gr_run(tmem + (uint32_t)bp.tmDZ, sDa, nZ, acc0, 47)) return false;
+        if (!gr_run(tmem + (uint32_t)bp.tmDZ, sPa, nZ, true, 48)) return false;
         tc_commit(gr_done);
         return true;
       };

@@ -70,6 +70,7 @@ static inline int make_bwd_plan(BwdPlan& b, const Plan& p, const char** why) {
     const long left = (long)limit - (long)slack - kBwdTailQ - (long)(b.nQr + b.nOc) * 16384;
     int nst = (int)(left / 16384);
     if (nst > 8) nst = 8;
+    if (nst > p.ring_cap) nst = p.ring_cap;
     if (nst < 2) { *why = "backward: shared memory too small for the q-side ring"; return 2; }
     b.q_nst = nst;
     b.q_smem = slack + kBwdTailQ + (size_t)(b.nQr + b.nOc + nst) * 16384;
@@ -79,6 +80,7 @@ static inline int make_bwd_plan(BwdPlan& b, const Plan& p, const char** why) {
     const long left = (long)limit - (long)slack - kBwdTailK - (long)(b.k_nres + 4) * 16384;
     int nst = (int)(left / 16384);
     if (nst > 8) nst = 8;
+    if (nst > p.ring_cap) nst = p.ring_cap;
     if (nst < 2) { *why = "backward: shared memory too small for the k-side ring"; return 2; }
     b.k_nst = nst;
     b.k_smem = slack + kBwdTailK + (size_t)(b.k_nres + 4 + nst) * 16384;

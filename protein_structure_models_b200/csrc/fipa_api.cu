@@ -42,6 +42,7 @@ struct fipa_handle {
   int trace_cta = -1;
   int pair_split = 1;
   int value_buffer = 1;
+  int ring_cap = 8;
   // TMA descriptors of the last call: they depend only on the workspace
   // address and the dims, so a loop over the same buffers encodes them once
   struct MapCache {
@@ -149,7 +150,7 @@ fipa_status ensure_maps(fipa_handle* h, const Plan& p, const fipa::Work& w, cons
 int plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
   const char* why = "";
   int rc = fipa::make_plan(p, d->B, d->N, d->H, d->D, d->Dv, d->P, d->Q, d->Cz, d->R, d->Cout,
-                           h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split, h->value_buffer);
+                           h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split, h->value_buffer, h->ring_cap);
   if (rc != 0) h->last_error = why;
   return rc;
 }
@@ -211,6 +212,10 @@ FIPA_API fipa_status fipa_create(fipa_handle** out, const fipa_dims* max_dims, f
   if (const char* env = std::getenv("FIPA_VALUE_BUFFER")) {
     const long v = std::strtol(env, nullptr, 10);
     h->value_buffer = v <= 0 ? 0 : (v >= 2 ? 2 : 1);
+  }
+  if (const char* env = std::getenv("FIPA_RING_STAGES")) {
+    const long v = std::strtol(env, nullptr, 10);
+    if (v >= 2 && v <= 8) h->ring_cap = (int)v;
   }
   if (const char* env = std::getenv("FIPA_TRACE_CTA")) {
     h->trace_cta = (int)std::strtol(env, nullptr, 10);

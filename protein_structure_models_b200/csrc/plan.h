@@ -95,6 +95,7 @@ struct Plan {
   int Pcols;          // TMEM columns holding P (64, or 128 for hi+lo)
   int tmemO;          // TMEM column of the O accumulator
   int nst;            // shared-memory ring stages of the core kernel
+  int ring_cap;       // most ring stages any kernel of this plan may use (tuning; default 8)
   // Value-buffer mode (bfloat16 inputs, when it fits): only QH and u hi of the
   // Qhat tile stay resident, the u lo chunks stream through the ring with the
   // key chunks, and each key tile's value chunks [VH | Z] land in a buffer of
@@ -134,7 +135,8 @@ struct Plan {
 // 0 = hi half only.  value_buffer: 1 = value-buffer mode where it fits and the
 // sample spans at least kVbufMinTiles key tiles, 2 = wherever it fits, 0 = off.
 static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, int Q, int Cz, int R,
-                            int Cout, int f32, const char** why, int pair_split = 1, int value_buffer = 1) {
+                            int Cout, int f32, const char** why, int pair_split = 1, int value_buffer = 1,
+                            int ring_cap = 8) {
   *why = "";
   if (B <= 0 || N <= 0 || H <= 0 || D <= 0 || Dv <= 0 || P <= 0 || Q <= 0 || Cz <= 0 || R <= 0 ||
       Cout <= 0) {
@@ -200,7 +202,9 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   size_t avail = limit - fixed - (size_t)(p.nQres + (p.vbuf ? p.nVB : 0)) * 16384;
   int nst = (int)(avail / 16384);
   if (nst > 8) nst = 8;
-  if (nst < 3) { *why = "shared memory too small for the ring"; return 2; }
+  if (nst > ring_cap) nst = ring_cap;
+  p.ring_cap = ring_cap;
+  if (nst < 2 || (nst < 3 && ring_cap >= 3)) { *why = "shared memory too small for the ring"; return 2; }
   p.nst = nst;
   const int nchunks = p.nQres + (p.vbuf ? p.nVB : 0) + nst;   // Qhat, value buffer, ring
   p.core_smem = fixed + (size_t)nchunks * 16384;
