@@ -267,9 +267,44 @@ fipa_status fipa_backward(fipa_handle* h,
                           void* workspace, size_t workspace_bytes,
                           void* stream);
 
+/* Training without the recompute: fipa_forward_train is fipa_forward (no
+ * attention output) that also keeps, in a workspace of
+ * fipa_backward_workspace_size() bytes, the state the backward needs (the
+ * lifted rows, the row statistics and the normalised aggregates of every row);
+ * fipa_backward_saved then takes the gradients from that state instead of
+ * recomputing the lift and the fused core.  Same arguments as fipa_forward /
+ * fipa_backward.  The workspace must not be written between the two calls, and
+ * both must get the same inputs and dims (not checked: the backward would use
+ * stale state).  The gradients equal fipa_backward's bit for bit.  bfloat16
+ * inputs only. */
+fipa_status fipa_forward_train(fipa_handle* h,
+                               const void* q, const void* k, const void* v,
+                               const void* q_pts, const void* k_pts, const void* v_pts,
+                               const void* rot, const void* trans,
+                               const void* z1, const void* z2, const void* Wb,
+                               const void* point_w_raw,
+                               const uint8_t* mask, const uint8_t* pair_mask,
+                               const void* w_out, const void* b_out, double eps,
+                               const fipa_dims* dims,
+                               float* out_update, float* out_local_points, float* out_lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+fipa_status fipa_backward_saved(fipa_handle* h,
+                                const void* q, const void* k, const void* v,
+                                const void* q_pts, const void* k_pts, const void* v_pts,
+                                const void* rot, const void* trans,
+                                const void* z1, const void* z2, const void* Wb,
+                                const void* point_w_raw,
+                                const uint8_t* mask, const uint8_t* pair_mask,
+                                const void* w_out, const void* b_out, double eps,
+                                const fipa_dims* dims,
+                                const float* d_update, const float* d_local_points,
+                                const fipa_grads* grads,
+                                void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Device time in milliseconds of each stage of the most recent fipa_backward
- * recorded with stage timing on (fipa_enable_stage_timing), in launch order:
- * [0] recompute (lift and fused core), [1] cotangent preparation (d_update @
+ * or fipa_backward_saved recorded with stage timing on (fipa_enable_stage_timing),
+ * in launch order: [0] recompute (lift and fused core; about 0 when saved), [1] cotangent preparation (d_update @
  * w_out^T and the per-residue dO rows), [2] q-side kernel (dS, dQhat), [3]
  * k-side kernel (dKhat, dVhat, dz2), [4] chain rule through frames and
  * factors and the weight gradients.  Waits for that call's last event. */

@@ -372,7 +372,7 @@ static fipa_status forward_impl(fipa_handle* h, const void* q, const void* k, co
                                 const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
                                 const void* b_out, double eps, const fipa_dims* dims, int row0, int row1,
                                 float* out_update, float* out_local_points, float* out_attention, float* out_lse,
-                                void* workspace, size_t workspace_bytes, void* stream) {
+                                void* workspace, size_t workspace_bytes, void* stream, float* osave = nullptr) {
   if (h == nullptr) return FIPA_ERR_INVALID_ARG;
   h->last_error.clear();
   if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
@@ -438,7 +438,7 @@ static fipa_status forward_impl(fipa_handle* h, const void* q, const void* k, co
   mark(0);
   if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
   mark(1);
-  if ((e = fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s)) != cudaSuccess)
+  if ((e = fipa::launch_core(p, in, w, out, tmQ, tmKH, tmVH, tmZ, ctl, s, osave)) != cudaSuccess)
     return cuda_fail(h, "core launch", e);
   mark(2);
   if ((e = fipa::launch_out_proj(p, in, w, out, tmA, tmB, ctl, s)) != cudaSuccess)
@@ -493,13 +493,13 @@ FIPA_API fipa_status fipa_backward_workspace_size(const fipa_handle* hc, const f
   return FIPA_OK;
 }
 
-FIPA_API fipa_status fipa_backward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
-                                   const void* k_pts, const void* v_pts, const void* rot, const void* trans,
-                                   const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
-                                   const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
-                                   const void* b_out, double eps, const fipa_dims* dims, const float* d_update,
-                                   const float* d_local_points, const fipa_grads* grads, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                 const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                 const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                 const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                 const void* b_out, double eps, const fipa_dims* dims, const float* d_update,
+                                 const float* d_local_points, const fipa_grads* grads, void* workspace,
+                                 size_t workspace_bytes, void* stream, bool recompute) {
   if (h == nullptr) return FIPA_ERR_INVALID_ARG;
   h->last_error.clear();
   if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
@@ -583,15 +583,67 @@ FIPA_API fipa_status fipa_backward(fipa_handle* h, const void* q, const void* k,
     cudaEventRecordWithFlags(m->h->bev[k], m->s, m->flags);
   };
   if (rec) mark(&mk, 0);
-  // recompute: the lift, and the core saving the normalised aggregates
-  if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
-  if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
-    return cuda_fail(h, "core launch", e);
+  if (recompute) {
+    // recompute: the lift, and the core saving the normalised aggregates
+    if ((e = fipa::launch_prologue(p, in, w, s)) != cudaSuccess) return cuda_fail(h, "prologue launch", e);
+    if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
+      return cuda_fail(h, "core launch", e);
+  }
   if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, ctl, s,
                                  rec ? +mark : nullptr, &mk)) != cudaSuccess)
     return cuda_fail(h, "backward launch", e);
   h->bwd_timed_call = rec;
   return FIPA_OK;
+}
+
+FIPA_API fipa_status fipa_backward(fipa_handle* h, const void* q, const void* k, const void* v, const void* q_pts,
+                                   const void* k_pts, const void* v_pts, const void* rot, const void* trans,
+                                   const void* z1, const void* z2, const void* Wb, const void* point_w_raw,
+                                   const uint8_t* mask, const uint8_t* pair_mask, const void* w_out,
+                                   const void* b_out, double eps, const fipa_dims* dims, const float* d_update,
+                                   const float* d_local_points, const fipa_grads* grads, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return backward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
+                       w_out, b_out, eps, dims, d_update, d_local_points, grads, workspace, workspace_bytes, stream,
+                       true);
+}
+
+FIPA_API fipa_status fipa_backward_saved(fipa_handle* h, const void* q, const void* k, const void* v,
+                                         const void* q_pts, const void* k_pts, const void* v_pts, const void* rot,
+                                         const void* trans, const void* z1, const void* z2, const void* Wb,
+                                         const void* point_w_raw, const uint8_t* mask, const uint8_t* pair_mask,
+                                         const void* w_out, const void* b_out, double eps, const fipa_dims* dims,
+                                         const float* d_update, const float* d_local_points,
+                                         const fipa_grads* grads, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  return backward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask,
+                       w_out, b_out, eps, dims, d_update, d_local_points, grads, workspace, workspace_bytes, stream,
+                       false);
+}
+
+FIPA_API fipa_status fipa_forward_train(fipa_handle* h, const void* q, const void* k, const void* v,
+                                        const void* q_pts, const void* k_pts, const void* v_pts, const void* rot,
+                                        const void* trans, const void* z1, const void* z2, const void* Wb,
+                                        const void* point_w_raw, const uint8_t* mask, const uint8_t* pair_mask,
+                                        const void* w_out, const void* b_out, double eps, const fipa_dims* dims,
+                                        float* out_update, float* out_local_points, float* out_lse, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (h == nullptr) return FIPA_ERR_INVALID_ARG;
+  if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
+  if (h->dtype != FIPA_BF16) return fail(h, FIPA_ERR_UNSUPPORTED, "the backward pass supports bfloat16 inputs only");
+  Plan p;
+  const int rc = plan_for(h, dims, p);
+  if (rc == 1) return FIPA_ERR_INVALID_ARG;
+  if (rc == 2) return FIPA_ERR_UNSUPPORTED;
+  fipa::BwdPlan bp;
+  const char* why = "";
+  if (fipa::make_bwd_plan(bp, p, &why) != 0) return fail(h, FIPA_ERR_UNSUPPORTED, why);
+  if (workspace == nullptr || workspace_bytes < bp.total)
+    return fail(h, FIPA_ERR_WORKSPACE, "training workspace needs " + std::to_string(bp.total) + " bytes");
+  float* osave = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + bp.off_osave);
+  return forward_impl(h, q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, mask, pair_mask, w_out,
+                      b_out, eps, dims, 0, -1, out_update, out_local_points, nullptr, out_lse, workspace,
+                      workspace_bytes, stream, osave);
 }
 
 FIPA_API fipa_status fipa_backward_stage_times(fipa_handle* h, float* ms, int n) {

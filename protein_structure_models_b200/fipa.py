@@ -95,6 +95,11 @@ def load_library():
     lib.fipa_backward.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double, ctypes.POINTER(FipaDims)] \
         + [vp, vp, ctypes.POINTER(FipaGrads), vp, sz, vp]
     lib.fipa_backward.restype = c_int
+    lib.fipa_backward_saved.argtypes = lib.fipa_backward.argtypes
+    lib.fipa_backward_saved.restype = c_int
+    lib.fipa_forward_train.argtypes = [vp] + [vp] * 12 + [vp, vp] + [vp, vp, ctypes.c_double,
+                                                                      ctypes.POINTER(FipaDims)] + [vp] * 3 + [vp, sz, vp]
+    lib.fipa_forward_train.restype = c_int
     lib.fipa_backward_stage_times.argtypes = [vp, ctypes.POINTER(ctypes.c_float), c_int]
     lib.fipa_backward_stage_times.restype = c_int
     lib.fipa_knn_distogram.argtypes = [c_int, vp, vp, c_int, c_int, c_int, vp, c_int, vp, vp, vp, vp, vp]
@@ -239,11 +244,34 @@ class Fipa:
         self._check(self.lib.fipa_backward_workspace_size(self.handle, ctypes.byref(d), ctypes.byref(n)))
         return int(n.value)
 
+    def forward_train(self, inp: dict, workspace: torch.Tensor, eps: float = 1e-8, out: Optional[dict] = None,
+                      want_lse: bool = False, stream: Optional[torch.cuda.Stream] = None) -> dict:
+        """fipa_forward_train: the forward, keeping in `workspace` (backward-sized)
+        the state backward(..., saved=True) uses instead of a recompute."""
+        dev = torch.device("cuda", self.device)
+        dims = self.dims_of(inp)
+        B, N, H, Q, Cout = dims["B"], dims["N"], dims["H"], dims["Q"], dims["Cout"]
+        if out is None:
+            out = {"update": torch.empty((B, N, Cout), dtype=torch.float32, device=dev),
+                   "local_points": torch.empty((B, N, H, Q, 3), dtype=torch.float32, device=dev)}
+            if want_lse:
+                out["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        d = make_dims(**dims)
+        self._check(self.lib.fipa_forward_train(
+            self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]), _ptr(inp.get("pair_mask")),
+            _ptr(inp["w_out"]), _ptr(inp["b_out"]), float(eps), ctypes.byref(d), _ptr(out["update"]),
+            _ptr(out["local_points"]), _ptr(out.get("lse")), _ptr(workspace), ctypes.c_size_t(workspace.numel()),
+            ctypes.c_void_p(s.cuda_stream)))
+        return out
+
     def backward(self, inp: dict, d_update: torch.Tensor, d_local: Optional[torch.Tensor] = None,
                  eps: float = 1e-8, workspace: Optional[torch.Tensor] = None, grads: Optional[dict] = None,
-                 stream: Optional[torch.cuda.Stream] = None) -> dict:
+                 stream: Optional[torch.cuda.Stream] = None, saved: bool = False) -> dict:
         """fipa_backward: float32 gradients of <d_update, update> + <d_local, local_points>
-        for every floating input, keyed like the inputs (see workloads.make_inputs)."""
+        for every floating input, keyed like the inputs (see workloads.make_inputs).
+        saved=True: fipa_backward_saved, from the state a forward_train call left in
+        `workspace` (no recompute)."""
         dev = torch.device("cuda", self.device)
         for k in INPUT_KEYS + ("w_out", "b_out"):
             t = inp[k]
@@ -261,7 +289,10 @@ class Fipa:
         gs = FipaGrads(*[grads[self.GRAD_KEYS[f]].data_ptr() for f in GRAD_FIELDS])
         s = stream if stream is not None else torch.cuda.current_stream(dev)
         d = make_dims(**dims)
-        st = self.lib.fipa_backward(self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]),
+        if saved and workspace is None:
+            raise ValueError("saved=True needs the workspace of a forward_train call")
+        fn = self.lib.fipa_backward_saved if saved else self.lib.fipa_backward
+        st = fn(self.handle, *[_ptr(inp[k]) for k in INPUT_KEYS], _ptr(inp["mask"]),
                                     _ptr(inp.get("pair_mask")), _ptr(inp["w_out"]), _ptr(inp["b_out"]),
                                     float(eps), ctypes.byref(d), _ptr(d_update), _ptr(d_local), ctypes.byref(gs),
                                     _ptr(workspace), ctypes.c_size_t(workspace.numel()),

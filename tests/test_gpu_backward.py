@@ -150,3 +150,24 @@ def test_backward_stage_times(handle):
         handle.enable_stage_timing(False)
     assert list(st) == ["recompute", "prep", "q_side", "k_side", "chain"]
     assert all(v > 0.0 for v in st.values()), st
+
+
+def test_forward_train_and_saved_backward(handle):
+    """fipa_forward_train gives fipa_forward's outputs, and fipa_backward_saved
+    (no recompute) gives fipa_backward's gradients, both bit for bit."""
+    inp = workloads.make_inputs(workloads.workload(1).with_(B=2))
+    dev = to_device(inp, "bf16")
+    du, dl = _cotangents(inp, 9)
+    d_update = torch.from_numpy(du).float().cuda().contiguous()
+    d_local = torch.from_numpy(dl).float().cuda().contiguous()
+    ref_fwd = handle.forward(dev, eps=inp["eps"], want_lse=True)
+    ref_bwd = handle.backward(dev, d_update, d_local, eps=inp["eps"])
+    ws = torch.empty(handle.backward_workspace_size(handle.dims_of(dev)), dtype=torch.uint8, device="cuda")
+    fwd = handle.forward_train(dev, ws, eps=inp["eps"], want_lse=True)
+    bwd = handle.backward(dev, d_update, d_local, eps=inp["eps"], workspace=ws, saved=True)
+    handle.sync_status()
+    torch.cuda.synchronize()
+    for k in ("update", "local_points", "lse"):
+        assert torch.equal(torch.nan_to_num(fwd[k], nan=7.0), torch.nan_to_num(ref_fwd[k], nan=7.0)), k
+    for k in ref_bwd:
+        assert torch.equal(bwd[k], ref_bwd[k]), k
