@@ -35,6 +35,7 @@ HARNESS = r"""
 #include <cstdio>
 #include <cstdlib>
 #include "plan.h"
+#include "bwd_plan.h"
 using namespace fipa;
 int main(int argc, char** argv) {
   int v[11];
@@ -58,6 +59,22 @@ int main(int argc, char** argv) {
     printf(", \"offs\": [");
     for (int i = 0; i < 15; ++i) printf("%s%zu", i ? ", " : "", offs[i]);
     printf("]");
+    BwdPlan b; const char* bwhy = "";
+    const int brc = make_bwd_plan(b, p, &bwhy);
+    printf(", \"bwd\": {\"rc\": %d, \"why\": \"%s\"", brc, bwhy);
+    if (brc == 0) {
+      printf(", \"q_smem\": %zu, \"k_smem\": %zu, \"q_nst\": %d, \"k_nst\": %d, \"nQr\": %d, \"nOc\": %d, \"k_nres\": %d",
+             b.q_smem, b.k_smem, b.q_nst, b.k_nst, b.nQr, b.nOc, b.k_nres);
+      printf(", \"tmDS\": %d, \"tmDQ\": %d, \"tmDK\": %d, \"tmDV\": %d, \"tmDZ\": %d, \"Vw\": %d, \"Kr\": %d, \"Kk\": %d, \"Fp\": %d",
+             b.tmDS, b.tmDQ, b.tmDK, b.tmDV, b.tmDZ, b.Vw, b.Kr, b.Kk, b.Fp);
+      const size_t bo[] = {b.off_lp, b.off_osave, b.off_dfeat, b.off_featp, b.off_dO, b.off_dvec, b.off_rloc,
+                           b.off_dz1u, b.off_qres, b.off_du, b.off_kres, b.off_dz2h, b.off_dwpart, b.off_wbpart,
+                           b.off_gpart, b.total};
+      printf(", \"offs\": [");
+      for (int i = 0; i < 16; ++i) printf("%s%zu", i ? ", " : "", bo[i]);
+      printf("]");
+    }
+    printf("}");
   }
   printf("}\n");
   return 0;
@@ -141,3 +158,32 @@ def test_mode_choices(plans):
         assert p["row0"] == 0 and p["row1"] == CASES[name][1], name   # full row range by default
         assert p["nT"] == (CASES[name][1] + 127) // 128, name
         assert p["lift_ctas"] == (CASES[name][1] + p["lift_res"] - 1) // p["lift_res"], name
+
+
+def test_backward_plan_budgets_and_layout(plans):
+    """The backward kernels' shared memory (<= 227 KB with the ring), tensor
+    memory (S/dP + dS + dQhat, and S^T/dP^T + dK + dV + dz2, each <= 512
+    columns) and the backward workspace regions (after the forward's,
+    256-byte aligned, in order) for every supported bfloat16 shape; float32
+    shapes are refused."""
+    for name, p in _ok(plans).items():
+        b = p["bwd"]
+        if CASES[name][10] == 1:
+            assert b["rc"] == 2 and "bfloat16" in b["why"], name
+            continue
+        assert b["rc"] == 0, (name, b["why"])
+        assert b["q_smem"] <= 232448 and b["k_smem"] <= 232448, name
+        assert b["q_nst"] >= 2 and b["k_nst"] >= 2, name
+        assert b["tmDQ"] + 64 * b["nQr"] <= 512 and b["tmDS"] + 64 <= b["tmDQ"], name
+        assert b["tmDZ"] + 64 * p["nZ"] <= 512 and b["tmDK"] >= 128, name
+        assert b["Vw"] == 64 * b["nOc"] and b["nOc"] == p["VHp"] // 64 + p["nZ"], name   # dO = [head | pair]
+        D, P, Dv, Q = CASES[name][3], CASES[name][5], CASES[name][4], CASES[name][6]
+        assert b["Kr"] >= D + 3 * P + 5 and b["Kk"] >= D + 3 * P + 4 + Dv + 3 * Q, name
+        assert b["Fp"] % 64 == 0 and b["Fp"] >= p["F"] + 1, name
+        offs = b["offs"]
+        assert offs[0] >= p["offs"][-1], name                  # after the forward's workspace
+        for a, c in zip(offs, offs[1:]):
+            assert a % 256 == 0 and a <= c, name
+    # the protein-batch and length-sweep widths use every tensor-memory column on both sides
+    b = plans["w3-16384"]["bwd"]
+    assert b["tmDQ"] + 64 * b["nQr"] == 512 and b["tmDZ"] + 64 * plans["w3-16384"]["nZ"] == 512
