@@ -171,3 +171,23 @@ def test_forward_train_and_saved_backward(handle):
         assert torch.equal(torch.nan_to_num(fwd[k], nan=7.0), torch.nan_to_num(ref_fwd[k], nan=7.0)), k
     for k in ref_bwd:
         assert torch.equal(bwd[k], ref_bwd[k]), k
+
+
+def test_backward_value_buffer_recompute(handle):
+    """A 1024-residue chain (8 key tiles: the recompute's core runs in
+    value-buffer mode) at reduced widths so the dense fp64 oracle stays small."""
+    wl = workloads.Workload("grad-vb", 9, B=1, N=1024, H=2, D=16, Dv=16, P=4, Q=8, Cz=32, R=2, Cout=32,
+                            dtype="bf16", frames="walk", t_scale=3.8)
+    check_grads(handle, workloads.make_inputs(wl, seed=21))
+
+
+def test_backward_single_half_pair_operand(monkeypatch):
+    """FIPA_PAIR_SPLIT=0: the pair-bias operand as one fp16 half (the backward
+    kernels' single-half branch)."""
+    from protein_structure_models_b200 import Fipa
+    monkeypatch.setenv("FIPA_PAIR_SPLIT", "0")
+    h = Fipa("bf16", 0)
+    try:
+        check_grads(h, _custom(23, N=200))
+    finally:
+        h.close()
