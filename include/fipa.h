@@ -230,9 +230,9 @@ typedef struct {
 } fipa_grads;
 
 /* Bytes of device workspace fipa_backward needs for `dims` (O(B*N): the
- * forward's workspace plus the backward's per-residue buffers).  Pure host
- * arithmetic.  FIPA_ERR_UNSUPPORTED for float32 inputs and for widths beyond
- * the backward kernels' tensor-memory or shared-memory budget. */
+ * recompute's workspace plus the backward's per-residue buffers).  Pure host
+ * arithmetic.  FIPA_ERR_UNSUPPORTED for widths beyond the backward kernels'
+ * tensor-memory or shared-memory budget. */
 fipa_status fipa_backward_workspace_size(const fipa_handle* h, const fipa_dims* dims,
                                          size_t* bytes);
 
@@ -250,9 +250,11 @@ fipa_status fipa_backward_workspace_size(const fipa_handle* h, const fipa_dims* 
  * also keeps the normalised aggregates of every row) inside the workspace, so
  * it needs no state from an earlier fipa_forward.  Rows with an empty
  * neighbourhood have constant (zero) outputs and pass no gradient back.
- * bfloat16 inputs only (FIPA_ERR_UNSUPPORTED otherwise).  Allocates nothing,
- * does not synchronise; kernels run on `stream`.  Deterministic: every sum is
- * taken in a fixed order. */
+ * Every product runs on fp16 tensor-core operands with fp32 accumulation, for
+ * bfloat16 and float32 inputs alike (float32 inputs are recomputed in the
+ * bfloat16 lifted layout); the gradients' normwise error is of the order of
+ * 1e-3.  Allocates nothing, does not synchronise; kernels run on `stream`.
+ * Deterministic: every sum is taken in a fixed order. */
 fipa_status fipa_backward(fipa_handle* h,
                           const void* q, const void* k, const void* v,
                           const void* q_pts, const void* k_pts, const void* v_pts,
@@ -276,7 +278,7 @@ fipa_status fipa_backward(fipa_handle* h,
  * fipa_backward.  The workspace must not be written between the two calls, and
  * both must get the same inputs and dims (not checked: the backward would use
  * stale state).  The gradients equal fipa_backward's bit for bit.  bfloat16
- * inputs only. */
+ * inputs only (FIPA_ERR_UNSUPPORTED otherwise). */
 fipa_status fipa_forward_train(fipa_handle* h,
                                const void* q, const void* k, const void* v,
                                const void* q_pts, const void* k_pts, const void* v_pts,

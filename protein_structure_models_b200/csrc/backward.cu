@@ -61,15 +61,16 @@ struct BwdArgs {
   unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ float ldb(const void* p, size_t i) {
-  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
+// An input value as float: float32 or bfloat16 inputs (Plan::in_f32).
+__device__ __forceinline__ float ldi(const void* p, size_t i, int f32) {
+  return f32 ? static_cast<const float*>(p)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
 }
 
 // ------------------------------------------------------------------ SIMT GEMMs
 // dfeat[m, n] = sum_k dupd[m, k] w[n, k]: the cotangent of the features,
 // d_update @ w_out^T (M = B*N rows, N = F features, K = Cout).
-__global__ void __launch_bounds__(256) bwd_dfeat_kernel(const float* __restrict__ A, const __nv_bfloat16* __restrict__ W,
-                                                        float* __restrict__ C, int M, int N, int K) {
+__global__ void __launch_bounds__(256) bwd_dfeat_kernel(const float* __restrict__ A, const void* __restrict__ W,
+                                                        int w_f32, float* __restrict__ C, int M, int N, int K) {
   __shared__ __align__(16) float As[32][68];
   __shared__ __align__(16) float Ws[32][68];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -83,7 +84,7 @@ __global__ void __launch_bounds__(256) bwd_dfeat_kernel(const float* __restrict_
     for (int e = threadIdx.x; e < 64 * 32; e += 256) {
       const int r = e >> 5, kk = e & 31, k = k0 + kk;
       As[kk][r] = (m0 + r < M && k < K) ? A[(size_t)(m0 + r) * K + k] : 0.f;
-      Ws[kk][r] = (n0 + r < N && k < K) ? __bfloat162float(W[(size_t)(n0 + r) * K + k]) : 0.f;
+      Ws[kk][r] = (n0 + r < N && k < K) ? ldi(W, (size_t)(n0 + r) * K + k, w_f32) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -204,8 +205,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     return;
   }
   for (int e = tid; e < F; e += 256) df[e] = a.dfeat[bi * F + e];
-  if (tid < 9) Rt[tid] = ldb(a.rot, bi * 9 + tid);
-  else if (tid < 12) Rt[tid] = ldb(a.trans, bi * 3 + tid - 9);
+  if (tid < 9) Rt[tid] = ldi(a.rot, bi * 9 + tid, a.p.in_f32);
+  else if (tid < 12) Rt[tid] = ldi(a.trans, bi * 3 + tid - 9, a.p.in_f32);
   __syncthreads();
   const float* R = Rt;
   const float* t = Rt + 9;
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
             x = sdG[h * 3 * Q + c - p.Dv8 - p.Q38];       // second copy: meets g' lo, not part of D
           } else if (c >= p.VHp && c < p.VHp + RCz) {
             const int rc = c - p.VHp, cc = rc % Cz;
-            x = ldb(a.z1, bi * RCz + rc) * df[pairblk + h * Cz + cc];
+            x = ldi(a.z1, bi * RCz + rc, a.p.in_f32) * df[pairblk + h * Cz + cc];
             o = Oh[Dv + 3 * Q + rc];
           }
           xv[u] = x;
@@ -316,7 +317,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     const int h = e / Cz, c = e - h * Cz;
     const float* U = a.osave + (bi * H + h) * (size_t)bp.Osw + Dv + 3 * Q;
     float s = 0.f;
-    for (int r = 0; r < p.R; ++r) s = fmaf(ldb(a.z1, bi * RCz + r * Cz + c), U[r * Cz + c], s);
+    for (int r = 0; r < p.R; ++r) s = fmaf(ldi(a.z1, bi * RCz + r * Cz + c, a.p.in_f32), U[r * Cz + c], s);
     fr[pairblk + e] = s;
   }
   for (int e = F + tid; e < bp.Fp; e += 256) fr[e] = e == F ? 1.f : 0.f;
@@ -331,7 +332,7 @@ __device__ __forceinline__ void bwd_drain_wait(uint64_t* bar, uint32_t parity, u
   }
 }
 
-__device__ __forceinline__ float bwd_raw(const BwdArgs& a, int h) { return ldb(a.raw, h); }
+__device__ __forceinline__ float bwd_raw(const BwdArgs& a, int h) { return ldi(a.raw, h, a.p.in_f32); }
 
 // The TMA ring shared by the producer and the MMA thread of both kernels.
 struct Ring {
@@ -1318,8 +1319,8 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
   for (int r = tid; r < nres; r += blockDim.x) {
     const int bi = bi0 + r, b = bi / N, i = bi - b * N;
     float* f = frm + r * 16;
-    for (int e = 0; e < 9; ++e) f[e] = ldb(a.rot, (size_t)bi * 9 + e);
-    for (int e = 0; e < 3; ++e) f[9 + e] = ldb(a.trans, (size_t)bi * 3 + e);
+    for (int e = 0; e < 9; ++e) f[e] = ldi(a.rot, (size_t)bi * 9 + e, a.p.in_f32);
+    for (int e = 0; e < 3; ++e) f[9 + e] = ldi(a.trans, (size_t)bi * 3 + e, a.p.in_f32);
     const float4 o = a.orig[(size_t)b * p.nG + i / kGroup];
     f[12] = o.x; f[13] = o.y; f[14] = o.z;
   }
@@ -1366,8 +1367,8 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
     for (int pp = 0; pp < P; ++pp) {
       float xq[3], xk[3], ap[3], bpp[3], da[3], db[3];
       for (int c = 0; c < 3; ++c) {
-        xq[c] = ldb(a.q_pts, (bih * P + pp) * 3 + c);
-        xk[c] = ldb(a.k_pts, (bih * P + pp) * 3 + c);
+        xq[c] = ldi(a.q_pts, (bih * P + pp) * 3 + c, a.p.in_f32);
+        xk[c] = ldi(a.k_pts, (bih * P + pp) * 3 + c, a.p.in_f32);
       }
 #pragma unroll
       for (int rr = 0; rr < 3; ++rr) {
@@ -1387,7 +1388,7 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
     for (int q = 0; q < Q; ++q) {
       float xv[3], dg[3];
       for (int c = 0; c < 3; ++c) {
-        xv[c] = ldb(a.v_pts, (bih * Q + q) * 3 + c);
+        xv[c] = ldi(a.v_pts, (bih * Q + q) * 3 + c, a.p.in_f32);
         dg[c] = kr[D + 3 * P + 4 + Dv + 3 * q + c];
       }
       frame_back(xv, dg, a.g.v_pts + (bih * Q + q) * 3);
@@ -1420,7 +1421,7 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
     float s1 = a.dz1u[(size_t)bi * RCz + rc], s2 = 0.f;
     for (int h = 0; h < H; ++h) {
       const size_t idx = ((size_t)b * H + h) * N + i;
-      s1 = fmaf(a.du[idx * RCz + rc], ldb(a.Wb, (size_t)c * H + h) * kInvSqrt3, s1);
+      s1 = fmaf(a.du[idx * RCz + rc], ldi(a.Wb, (size_t)c * H + h, a.p.in_f32) * kInvSqrt3, s1);
       s2 += a.dz2h[idx * RCz + rc];
     }
     a.g.z1[(size_t)bi * RCz + rc] = s1;
@@ -1433,7 +1434,7 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
       const int bi = bi0 + r, b = bi / N, i = bi - b * N;
       const size_t idx = ((size_t)b * H + h) * N + i;
       for (int rr = 0; rr < p.R; ++rr)
-        s = fmaf(a.du[idx * RCz + rr * Cz + c], ldb(a.z1, (size_t)bi * RCz + rr * Cz + c), s);
+        s = fmaf(a.du[idx * RCz + rr * Cz + c], ldi(a.z1, (size_t)bi * RCz + rr * Cz + c, a.p.in_f32), s);
     }
     a.wbpart[(size_t)blockIdx.x * Cz * H + e] = s * kInvSqrt3;
   }
@@ -1505,7 +1506,7 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   cudaError_t e;
   stage(1);
   bwd_dfeat_kernel<<<dim3(cdiv(p.F, 64), cdiv(BN, 64)), 256, 0, s>>>(
-      io.d_update, static_cast<const __nv_bfloat16*>(in.w_out), a.dfeat, BN, p.F, p.Cout);
+      io.d_update, in.w_out, p.in_f32, a.dfeat, BN, p.F, p.Cout);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t psm = bwd_prep_smem(p);
   if (psm > 48 * 1024) {

@@ -80,7 +80,7 @@ constexpr int kTiles = 5120;       // uint16 key-tile list (<= 1024 entries)
 constexpr int kKpBuf = 7168;       // fp32 key points of two key tiles (float32-input mode)
 
 __device__ __forceinline__ float load_raw(const CoreArgs& a, int h) {
-  return a.p.f32 ? static_cast<const float*>(a.raw)[h]
+  return a.p.in_f32 ? static_cast<const float*>(a.raw)[h]
                  : __bfloat162float(static_cast<const __nv_bfloat16*>(a.raw)[h]);
 }
 
@@ -234,7 +234,7 @@ __device__ void write_features(const CoreArgs& a, size_t bi, bool empty, float* 
     for (int rr = 0; rr < p.R; ++rr) {
       float u = orow[p.VHp + rr * Cz + c];
       if (p.f32) u += orow[p.VHp + p.RC8 + rr * Cz + c];
-      acc = fmaf(ld_any(a.z1, bi * RCz + rr * Cz + c, p.f32), u, acc);
+      acc = fmaf(ld_any(a.z1, bi * RCz + rr * Cz + c, p.in_f32), u, acc);
     }
     return acc;
   });
@@ -259,7 +259,7 @@ __device__ __forceinline__ EpiLayout epi_layout(const Plan& p, const void* z1) {
   const uint32_t ring_end = (uint32_t)(p.nQres + (p.vbuf ? p.nVB : 0) + p.nst) * kChunkBytes;
   e.fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(z1) & 15) == 0;
   e.staged = e.fast_pair ? p.VHp : p.Ocols;
-  e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.f32 ? 4 : 2));
+  e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.in_f32 ? 4 : 2));
   e.z1_stride = e.z1_row_bytes + 16;
   const uint32_t o_bytes = (uint32_t)kTile * (e.staged + 1) * 4;
   e.z1_smem = e.fast_pair && (e.z1_row_bytes & 15) == 0 &&
@@ -836,9 +836,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int i = qt * kTile + wq * 32 + lane;
       const size_t bi = (size_t)b * N + (i < N ? i : 0);
 #pragma unroll
-      for (int e = 0; e < 9; ++e) rowR[e] = ld_any(a.rot, bi * 9 + e, p.f32);
+      for (int e = 0; e < 9; ++e) rowR[e] = ld_any(a.rot, bi * 9 + e, p.in_f32);
 #pragma unroll
-      for (int e = 0; e < 3; ++e) rowT[e] = ld_any(a.trans, bi * 3 + e, p.f32);
+      for (int e = 0; e < 3; ++e) rowT[e] = ld_any(a.trans, bi * 3 + e, p.in_f32);
       const EpiLayout el = epi_layout(p, a.z1);
       if (el.z1_smem && i < N) {
         const uint8_t* src = static_cast<const uint8_t*>(a.z1) + bi * el.z1_row_bytes;
@@ -946,7 +946,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             const size_t zoff = bi * RCz + (size_t)rr * Cz + c0;
             const size_t zrel = (size_t)rr * Cz + c0;
             float zv[32];
-            if (p.f32) {
+            if (p.in_f32) {
               const float4* z4 = el.z1_smem ? reinterpret_cast<const float4*>(zs) + zrel / 4
                                          : reinterpret_cast<const float4*>(static_cast<const float*>(a.z1) + zoff);
 #pragma unroll

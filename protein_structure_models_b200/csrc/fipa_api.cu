@@ -49,6 +49,7 @@ struct fipa_handle {
     bool valid = false;
     const void* ws = nullptr;
     fipa_dims dims{};
+    int sig[5] = {0, 0, 0, 0, 0};   // layout widths the maps were encoded for
     CUtensorMap Q, KH, VH, Z, A, B;
   } maps;
   // the backward's dO map, cached the same way
@@ -129,7 +130,9 @@ fipa_status ensure_maps(fipa_handle* h, const Plan& p, const fipa::Work& w, cons
                         const fipa_dims* dims) {
   const uint64_t BH = (uint64_t)p.B * p.H, N = (uint64_t)p.N, B = (uint64_t)p.B;
   fipa_handle::MapCache& mc = h->maps;
-  if (!mc.valid || mc.ws != workspace || std::memcmp(&mc.dims, dims, sizeof(fipa_dims)) != 0) {
+  const int sig[5] = {p.Kq, p.KHp, p.VHp, p.Zp, p.Kgp};
+  if (!mc.valid || mc.ws != workspace || std::memcmp(&mc.dims, dims, sizeof(fipa_dims)) != 0 ||
+      std::memcmp(mc.sig, sig, sizeof(sig)) != 0) {
     mc.valid = false;
     fipa_status st;
     if ((st = encode_rows(h, &mc.Q, w.Q, p.Kq, N, BH, 128, 3, "Qhat")) != FIPA_OK) return st;
@@ -142,6 +145,7 @@ fipa_status ensure_maps(fipa_handle* h, const Plan& p, const fipa::Work& w, cons
       return st;
     mc.ws = workspace;
     mc.dims = *dims;
+    std::memcpy(mc.sig, sig, sizeof(sig));
     mc.valid = true;
   }
   return FIPA_OK;
@@ -153,6 +157,21 @@ int plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
                            h->dtype == FIPA_F32 ? 1 : 0, &why, h->pair_split, h->value_buffer, h->ring_cap);
   if (rc != 0) h->last_error = why;
   return rc;
+}
+
+// The forward plan the backward recomputes with: the bfloat16 lifted layout
+// (fp16 products), reading the handle's input dtype.  float32 inputs are thus
+// differentiated at the backward's fp16-product precision.
+int bwd_plan_for(fipa_handle* h, const fipa_dims* d, Plan& p) {
+  const char* why = "";
+  int rc = fipa::make_plan(p, d->B, d->N, d->H, d->D, d->Dv, d->P, d->Q, d->Cz, d->R, d->Cout, 0, &why,
+                           h->pair_split, h->value_buffer, h->ring_cap);
+  if (rc != 0) {
+    h->last_error = why;
+    return rc;
+  }
+  p.in_f32 = h->dtype == FIPA_F32 ? 1 : 0;
+  return 0;
 }
 
 }  // namespace
@@ -483,7 +502,7 @@ FIPA_API fipa_status fipa_backward_workspace_size(const fipa_handle* hc, const f
   fipa_handle* h = const_cast<fipa_handle*>(hc);
   if (h == nullptr || dims == nullptr || bytes == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "null argument");
   Plan p;
-  const int rc = plan_for(h, dims, p);
+  const int rc = bwd_plan_for(h, dims, p);
   if (rc == 1) return FIPA_ERR_INVALID_ARG;
   if (rc == 2) return FIPA_ERR_UNSUPPORTED;
   fipa::BwdPlan bp;
@@ -503,9 +522,10 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
   if (h == nullptr) return FIPA_ERR_INVALID_ARG;
   h->last_error.clear();
   if (dims == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "dims is NULL");
-  if (h->dtype != FIPA_BF16) return fail(h, FIPA_ERR_UNSUPPORTED, "the backward pass supports bfloat16 inputs only");
+  if (h->dtype != FIPA_BF16 && !recompute)
+    return fail(h, FIPA_ERR_UNSUPPORTED, "the backward from saved state supports bfloat16 inputs only");
   Plan p;
-  const int rc = plan_for(h, dims, p);
+  const int rc = bwd_plan_for(h, dims, p);
   if (rc == 1) return FIPA_ERR_INVALID_ARG;
   if (rc == 2) return FIPA_ERR_UNSUPPORTED;
   if (h->has_max) {
@@ -520,9 +540,10 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
   const void* req[] = {q, k, v, q_pts, k_pts, v_pts, rot, trans, z1, z2, Wb, point_w_raw, w_out, b_out};
   const char* names[] = {"q", "k", "v", "q_pts", "k_pts", "v_pts", "rot", "trans", "z1", "z2", "Wb",
                          "point_w_raw", "w_out", "b_out"};
+  const size_t ies = h->dtype == FIPA_F32 ? 4 : 2;
   for (int i = 0; i < 14; ++i) {
     if (req[i] == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is NULL");
-    if (!aligned(req[i], 2)) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is misaligned");
+    if (!aligned(req[i], ies)) return fail(h, FIPA_ERR_INVALID_ARG, std::string(names[i]) + " is misaligned");
   }
   if (mask == nullptr) return fail(h, FIPA_ERR_INVALID_ARG, "mask is NULL");
   if (d_update == nullptr || !aligned(d_update, 4) || !aligned(d_local_points, 4))

@@ -72,7 +72,9 @@ static inline size_t rup_sz(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
 struct Plan {
   int B, N, H, D, Dv, P, Q, Cz, R, Cout, F;
-  int f32;            // 1: float32 inputs (hi/lo splits everywhere); 0: bfloat16 inputs
+  int f32;            // 1: float32 layout (hi/lo splits everywhere, fp32 distance); 0: bfloat16 layout
+  int in_f32;         // dtype of the inputs: 1 float32, 0 bfloat16 (== f32, except for the backward's
+                      // recompute of float32 inputs in the bfloat16 layout)
   int nT;             // tiles per sample
   // query rows computed by this forward, the same range in every sample: row0
   // a multiple of the 128-row tile, row1 a multiple of it or N (all keys are
@@ -146,6 +148,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.B = B; p.N = N; p.H = H; p.D = D; p.Dv = Dv; p.P = P; p.Q = Q; p.Cz = Cz; p.R = R; p.Cout = Cout;
   p.F = H * (Dv + 4 * Q + Cz);
   p.f32 = f32 ? 1 : 0;
+  p.in_f32 = p.f32;
   p.nT = cdiv(N, kTile);
   p.row0 = 0;
   p.row1 = N;

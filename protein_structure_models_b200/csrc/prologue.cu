@@ -456,11 +456,11 @@ cudaError_t launch_prologue(const Plan& p, const Inputs& in, const Work& w, cuda
   // one launch: the weight-preparation CTAs first, then B x lift_ctas lift CTAs
   PrologueArgs a{p, in, w};
   const unsigned grid = (unsigned)(p.wp_ctas + (size_t)p.B * p.lift_ctas);
-  const void* kfn = p.f32 ? reinterpret_cast<const void*>(fipa_lift_kernel<float>)
-                          : reinterpret_cast<const void*>(fipa_lift_kernel<__nv_bfloat16>);
+  const void* kfn = p.in_f32 ? reinterpret_cast<const void*>(fipa_lift_kernel<float>)
+                             : reinterpret_cast<const void*>(fipa_lift_kernel<__nv_bfloat16>);
   cudaError_t e = allow_max_smem(kfn);
   if (e != cudaSuccess) return e;
-  if (p.f32)
+  if (p.in_f32)
     fipa_lift_kernel<float><<<grid, kLiftThreads, p.lift_smem, s>>>(a);
   else
     fipa_lift_kernel<__nv_bfloat16><<<grid, kLiftThreads, p.lift_smem, s>>>(a);

@@ -3,7 +3,7 @@ backward oracle (oracle/backward.py: the vector-Jacobian product of the page's
 forward, "Invariant point attention (IPA)", Required behavior; the page's
 "Starter code" section grades the suite "including gradients").
 
-Tolerance (bfloat16 inputs; the derivation is in the design notes): for every
+Tolerance (fp16 products for bfloat16 and float32 inputs alike): for every
 gradient tensor, max |g - g_ref| <= GRAD_TOL * max |g_ref|, GRAD_TOL = 1e-2.
 The fp16 operands of the recomputed products and of dS carry 2^-11 relative
 rounding each; dS = P (dP - D) loses up to a few bits where dP is close to D;
@@ -124,7 +124,38 @@ def test_backward_deterministic(handle):
         assert np.array_equal(a[key], b[key]), key
 
 
-def test_backward_rejects_float32(handle):
+def test_backward_float32_inputs():
+    """float32 inputs: the recompute reads them in the bfloat16 lifted layout
+    (fp16 products), so the same 1e-2 normwise bound applies; the tiny float32
+    workload (masks, an empty pair row) and an odd-width ragged case."""
+    from protein_structure_models_b200 import Fipa
+    h = Fipa("f32", 0)
+    try:
+        for inp in (workloads.make_inputs(workloads.workload(0)), _custom_f32(31, N=129)):
+            du, dl = _cotangents(inp, 4)
+            dev = to_device(inp, "f32")
+            g = h.backward(dev, torch.from_numpy(du).float().cuda(), torch.from_numpy(dl).float().cuda(),
+                           eps=inp["eps"])
+            h.sync_status()
+            torch.cuda.synchronize()
+            got = {k: v.double().cpu().numpy() for k, v in g.items()}
+            ref = bw.ipa_vjp(inp, du, dl)
+            errs = {k: float(np.max(np.abs(got[k] - ref[k])) / max(1e-30, float(np.max(np.abs(ref[k])))))
+                    for k in bw.FLOAT_KEYS}
+            print({k: f"{v:.2e}" for k, v in errs.items()})
+            assert all(v <= GRAD_TOL for v in errs.values()), errs
+    finally:
+        h.close()
+
+
+def _custom_f32(seed, **kw):
+    base = dict(B=2, N=40, H=3, D=5, Dv=3, P=3, Q=5, Cz=7, R=3, Cout=20)
+    base.update(kw)
+    wl = workloads.Workload("edge32", 9, dtype="f32", frames="walk", t_scale=3.8, **base)
+    return workloads.make_inputs(wl, seed=seed)
+
+
+def test_saved_backward_rejects_float32():
     from protein_structure_models_b200 import Fipa
     from protein_structure_models_b200.fipa import FipaError
     h = Fipa("f32", 0)
@@ -133,7 +164,7 @@ def test_backward_rejects_float32(handle):
         dev = to_device(inp, "f32")
         du = torch.zeros((1, 32, 32), dtype=torch.float32, device="cuda")
         with pytest.raises(FipaError, match="UNSUPPORTED"):
-            h.backward(dev, du, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"))
+            h.backward(dev, du, workspace=torch.empty(1 << 20, dtype=torch.uint8, device="cuda"), saved=True)
     finally:
         h.close()
 
