@@ -280,12 +280,44 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, uint6
 // SPLIT: float32 inputs (3-way operands, P as hi + lo, exact point term).
 // VB: value-buffer mode (bfloat16 only): each key tile's value chunks [VH | Z]
 // land in a buffer of their own and the u lo chunks stream with the keys.
+// A query tile without a valid residue (the padding of a short sample): every
+// row has an empty neighbourhood, so only the outputs the full path leaves for
+// such rows are written (row statistics (-inf, 0), lse -inf, zero local points,
+// the row flag and the feature padding) and nothing is computed.  Out of line,
+// so the full path's code is unchanged.
+__device__ __noinline__ void core_masked_tile(float2* stats, float* lse, uint8_t* rowflag, __half* feat,
+                                              float* local_points, int N, int H, int Q, int Kg, int Kgp,
+                                              int qt, int h, int b) {
+  const int bh = b * H + h;
+  for (int r = threadIdx.x; r < kTile; r += blockDim.x) {
+    const int i = qt * kTile + r;
+    if (i >= N) continue;
+    const size_t bi = (size_t)b * N + i;
+    stats[(size_t)bh * N + i] = make_float2(-INFINITY, 0.f);
+    if (lse != nullptr) lse[(size_t)bh * N + i] = -INFINITY;
+    if (h == 0) {
+      rowflag[bi] = 0;
+      for (int c = Kg; c < Kgp; ++c) feat[bi * Kgp + c] = __float2half_rn(0.f);
+    }
+    float* lp = local_points + (bi * H + h) * (size_t)Q * 3;
+    for (int e = 0; e < 3 * Q; ++e) lp[e] = 0.f;
+  }
+}
+
 // SAVE: also store the normalised aggregates of every row (training recompute).
 template <bool SPLIT, bool VB, bool SAVE>
 __global__ void __launch_bounds__(256, 1)
 fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKH,
                  const __grid_constant__ CUtensorMap tmVH, const __grid_constant__ CUtensorMap tmZ,
                  const CoreArgs a) {
+  {
+    const int qt0 = blockIdx.x + a.p.row0 / kTile;
+    if (a.flag[(size_t)blockIdx.z * a.p.nT + qt0] == 0) {   // uniform over the CTA
+      core_masked_tile(a.stats, a.lse, a.rowflag, a.feat, a.local_points, a.p.N, a.p.H, a.p.Q, a.p.Kg, a.p.Kgp,
+                       qt0, blockIdx.y, blockIdx.z);
+      return;
+    }
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Plan& p = a.p;
