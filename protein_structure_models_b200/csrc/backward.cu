@@ -348,6 +348,28 @@ struct Ring {
   }
 };
 
+// Bit e: pair-mask entry first + e (stride `stride` bytes apart) allowed; 0 past
+// N.  Every load is issued unconditionally (an index past N reads entry 0) and
+// the results combine afterwards, so the 32 loads are in flight together.
+__device__ __forceinline__ uint32_t pair_bits32(const uint8_t* base, size_t stride, int first, int N) {
+  uint32_t v[32];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const int x = first + e;
+    v[e] = __ldg(base + (size_t)(x < N ? x : 0) * stride);
+  }
+  uint32_t bits = 0;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) bits |= (first + e < N && v[e] != 0u) ? (1u << e) : 0u;
+  return bits;
+}
+// The 128 bits of a tile, out of line: the loads' registers stay out of the
+// kernels' main loops (the pair mask is the uncommon case).
+__device__ __noinline__ uint4 pair_bits128(const uint8_t* base, size_t stride, int first, int N) {
+  return make_uint4(pair_bits32(base, stride, first, N), pair_bits32(base, stride, first + 32, N),
+                    pair_bits32(base, stride, first + 64, N), pair_bits32(base, stride, first + 96, N));
+}
+
 // ------------------------------------------------------------------ q side
 // One CTA per (query tile, head, sample), as the forward core.  Per key tile s:
 //   QK(s): S = Qhat Khat^T (u hi resident, u lo streamed with the z2 chunks)
@@ -667,10 +689,22 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         rc[t] = -g * ((float)p.P * (dx * dx + dy * dy + dz * dz) + 2.f * (dx * qv.x + dy * qv.y + dz * qv.z));
       }
       const float* ktw = ktbuf + (kb * 4 + wq) * kTile;
+      // a forbidden pair gets the logit -inf in a pass of its own, so that the
+      // loop below has no branch (absent or masked keys have kterm -inf already)
+      if (pmrow != nullptr) {
+        const uint4 b4 = pair_bits128(pmrow, 1, kt * kTile, N);
+        const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            sv[t][e] = ((bw[t] >> e) & 1u) ? sv[t][e] : __float_as_uint(-INFINITY);
+      }
+      const bool allow = invl > 0.f;
       uint32_t pk[2][32];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const float mb = invl > 0.f ? st.x - rc[t] * kLog2e : 0.f;
+        const float mb = allow ? st.x - rc[t] * kLog2e : 0.f;
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float pv[2];
@@ -678,11 +712,6 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           for (int u = 0; u < 2; ++u) {
             const int jl = t * 32 + e + u;
             const float x = __uint_as_float(sv[t][e + u]) + ktw[jl];
-            bool allow = invl > 0.f;
-            if (pmrow != nullptr) {
-              const int j = kt * kTile + jl;
-              allow = allow && j < N && pmrow[j] != 0;
-            }
             pv[u] = allow ? ex2_approx(fmaf(x, kLog2e, -mb)) * invl : 0.f;
           }
           pk[t >> 1][(t & 1) * 16 + e / 2] = pack_half2(pv[0], pv[1]);
@@ -800,12 +829,15 @@ bwd_q_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
 //   DPT(s): dP^T = Vhat dO^T into the same TMEM columns
 //   GR(s):  with P^T and dS^T (fp16, K-major) written to shared memory by the
 //           softmax warps: dK head += dS^T QH, dV head += P^T dO head,
-//           dz2 += dS^T u (hi and lo) + P^T dU, the B operands streamed again
+//           dz2 += dS^T u hi + P^T dU, the B operands streamed again (the u hi
+//           and dU rows as slices of 32 queries x every pair column, so that
+//           each landed slot feeds two MMAs of the full width N = 64 nZ)
 // issued as ST(0) DPT(0) [ST(s+1) GR(s) DPT(s+1)]....
 constexpr int kKBarFull = 0, kKBarEmpty = 64, kKBarRes = 128, kKBarStFull = 136, kKBarStRead = 144,
               kKBarDpFull = 152, kKBarDpRead = 160, kKBarPdsFull = 168, kKBarGrDone = 176, kKBarQdFull = 184,
               kKBarQdEmpty = 200, kKBarDrain = 216;
 constexpr int kKMisc = 256, kKOq = 512, kKQd = 1024, kKQdFloats = 9 * 128, kKTiles = 10240;
+constexpr int kSliceGroupBytes = 32 * 128;   // one 32-row x 64-column fp16 box (128-byte swizzle)
 
 __device__ __forceinline__ void zero_key_rows(const BwdArgs& a, int b, int h, int kt) {
   const Plan& p = a.p;
@@ -824,7 +856,8 @@ __device__ __forceinline__ void zero_key_rows(const BwdArgs& a, int b, int h, in
 __global__ void __launch_bounds__(256, 1)
 bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKH,
              const __grid_constant__ CUtensorMap tmVH, const __grid_constant__ CUtensorMap tmZ,
-             const __grid_constant__ CUtensorMap tmdO, const BwdArgs a) {
+             const __grid_constant__ CUtensorMap tmdO, const __grid_constant__ CUtensorMap tmQ32,
+             const __grid_constant__ CUtensorMap tmdO32, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Plan& p = a.p;
@@ -903,6 +936,8 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       tma_prefetch_desc(&tmVH);
       tma_prefetch_desc(&tmZ);
       tma_prefetch_desc(&tmdO);
+      tma_prefetch_desc(&tmQ32);
+      tma_prefetch_desc(&tmdO32);
       mbar_arrive_expect_tx(res_full, (uint32_t)(bp.k_nres * kChunkBytes));
       for (int c = 0; c < nKH; ++c) tma_load_3d(sK + c * kChunkBytes, &tmKH, res_full, c * kChunk, kt * kTile, bh);
       for (int c = 0; c < nZ; ++c)
@@ -928,15 +963,28 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
       auto push_dp = [&](int qt) {
         for (int c = 0; c < bp.nOc; ++c) push(&tmdO, c * kChunk, qt);
       };
-      // gradient products: QH, dO head, then the u hi and dU chunks each as one
-      // run of consecutive ring slots (the dz2 product uses u hi only: the lo
-      // half is 2^-12 of u, far below the gradient tolerance; the logits above
-      // are recomputed with both halves)
+      // one slot = 32 queries x the nZ 64-column groups from column col0, one
+      // 32-row box per group, 4 KB apart (a K slice of an N = 64 nZ operand)
+      auto push_slices = [&](const CUtensorMap* tm, int col0, int qt) {
+        for (int sl = 0; sl < kTile / 32; ++sl) {
+          if (!ok) return;
+          if (!mbar_wait(&empty[rg.st], rg.ph ^ 1u, wc, 41)) { ok = false; return; }
+          mbar_arrive_expect_tx(&full[rg.st], (uint32_t)(nZ * kSliceGroupBytes));
+          for (int c = 0; c < nZ; ++c)
+            tma_load_3d(rg.slot() + c * kSliceGroupBytes, tm, &full[rg.st], col0 + c * kChunk, qt * kTile + sl * 32,
+                        bh);
+          ++issued;
+          rg.next();
+        }
+      };
+      // gradient products: QH, dO head, then the u hi and dU slices (the dz2
+      // product uses u hi only: the lo half is 2^-12 of u, far below the
+      // gradient tolerance; the logits above are recomputed with both halves)
       auto push_gr = [&](int qt) {
         for (int c = 0; c < nKH; ++c) push(&tmQ, c * kChunk, qt);
         for (int c = 0; c < nVH; ++c) push(&tmdO, c * kChunk, qt);
-        for (int c = 0; c < nZ; ++c) push(&tmQ, (nKH + c) * kChunk, qt);
-        for (int c = 0; c < nZ; ++c) push(&tmdO, (nVH + c) * kChunk, qt);
+        push_slices(&tmQ32, nKH * kChunk, qt);
+        push_slices(&tmdO32, nVH * kChunk, qt);
       };
       push_st(tiles[0]);
       push_dp(tiles[0]);
@@ -1041,12 +1089,27 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         }
         return true;
       };
+      // dz2 += dS^T u hi + P^T dU: per slot of 32 queries, two K steps of one
+      // MMA over all 64 nZ columns (MN-major B, column groups 4 KB apart)
+      const uint32_t idZ = idesc_f16(128, 64 * nZ, 0, 1);
       auto mma_gr = [&](int s) -> bool {
         const bool acc0 = s > 0;
         if (!gr_run(tmem + (uint32_t)bp.tmDK, sDa, nKH, acc0, 45)) return false;
         if (!gr_run(tmem + (uint32_t)bp.tmDV, sPa, nVH, acc0, 46)) return false;
-        if (!gr_run(tmem + (uint32_t)bp.tmDZ, sDa, nZ, acc0, 47)) return false;
-        if (!gr_run(tmem + (uint32_t)bp.tmDZ, sPa, nZ, true, 48)) return false;
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t abase = part == 0 ? sDa : sPa;
+          for (int sl = 0; sl < kTile / 32; ++sl) {
+            const int st = take(part == 0 ? 47 : 48);
+            if (st < 0) return false;
+            const uint32_t bq = ringa + st * kChunkBytes;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk)
+              mma_ss(tmem + (uint32_t)bp.tmDZ, adesc(abase, 2 * sl + kk),
+                     desc_mnmajor_sw128(bq + kk * 2048, kSliceGroupBytes), idZ,
+                     (part > 0 || acc0 || sl > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&empty[st]);
+          }
+        }
         tc_commit(gr_done);
         return true;
       };
@@ -1149,6 +1212,18 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
         const float dx = oq[t].x - okj.x, dy = oq[t].y - okj.y, dz = oq[t].z - okj.z;
         ktm[t] = kv.x + 2.f * g * (dx * kv.y + dy * kv.z + dz * kv.w);
       }
+      // a forbidden pair gets the logit -inf in a pass of its own, so that the
+      // loop below has no branch (an absent key has kterm -inf already)
+      if (a.pair_mask != nullptr) {
+        const uint8_t* pmcol = a.pair_mask + (size_t)b * N * N + (jin ? j : 0);
+        const uint4 b4 = pair_bits128(pmcol, (size_t)N, qt * kTile, N);
+        const uint32_t bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            sv[t][e] = ((bw[t] >> e) & 1u) ? sv[t][e] : __float_as_uint(-INFINITY);
+      }
       uint32_t pk[2][32];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -1159,13 +1234,8 @@ bwd_k_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CU
           for (int u = 0; u < 2; ++u) {
             const int il = t * 32 + e + u;
             const float il_inv = ilw[il];
-            bool allow = il_inv > 0.f;
-            if (a.pair_mask != nullptr && allow) {
-              const int i = qt * kTile + il;
-              allow = jin && a.pair_mask[((size_t)b * N + i) * N + j] != 0;
-            }
             const float x = __uint_as_float(sv[t][e + u]) + ktm[t];
-            pv[u] = allow ? ex2_approx(fmaf(x, kLog2e, -mbw[il])) * il_inv : 0.f;
+            pv[u] = il_inv > 0.f ? ex2_approx(fmaf(x, kLog2e, -mbw[il])) * il_inv : 0.f;
           }
           pk[t >> 1][(t & 1) * 16 + e / 2] = pack_half2(pv[0], pv[1]);
         }
@@ -1471,7 +1541,8 @@ size_t bwd_chain_smem(const Plan& p) {
 
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s,
+                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const CUtensorMap& tmQ32,
+                            const CUtensorMap& tmdO32, const DeviceCtl& ctl, cudaStream_t s,
                             StageMark mark, void* mark_ctx) {
   auto stage = [&](int k) {
     if (mark != nullptr) mark(mark_ctx, k);
@@ -1521,7 +1592,7 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_k_kernel))) != cudaSuccess) return e;
   stage(3);
-  bwd_k_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.k_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, a);
+  bwd_k_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.k_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, tmQ32, tmdO32, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage(4);
   const size_t csm = bwd_chain_smem(p);

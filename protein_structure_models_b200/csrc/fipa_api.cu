@@ -52,12 +52,13 @@ struct fipa_handle {
     int sig[5] = {0, 0, 0, 0, 0};   // layout widths the maps were encoded for
     CUtensorMap Q, KH, VH, Z, A, B;
   } maps;
-  // the backward's dO map, cached the same way
+  // the backward's maps, cached the same way: dO with 128-row boxes, and Qhat
+  // and dO with 32-row boxes (the k side's slices of the pair columns)
   struct BwdMapCache {
     bool valid = false;
     const void* ws = nullptr;
     fipa_dims dims{};
-    CUtensorMap dO;
+    CUtensorMap dO, Q32, dO32;
   } bmaps;
 };
 
@@ -574,8 +575,10 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
   fipa_handle::BwdMapCache& bm = h->bmaps;
   if (!bm.valid || bm.ws != workspace || std::memcmp(&bm.dims, dims, sizeof(fipa_dims)) != 0) {
     bm.valid = false;
-    if ((mst = encode_rows(h, &bm.dO, ws + bp.off_dO, bp.Vw, (uint64_t)p.N, (uint64_t)p.B * p.H, 128, 3, "dO")) !=
-        FIPA_OK)
+    const uint64_t BH = (uint64_t)p.B * p.H;
+    if ((mst = encode_rows(h, &bm.dO, ws + bp.off_dO, bp.Vw, (uint64_t)p.N, BH, 128, 3, "dO")) != FIPA_OK ||
+        (mst = encode_rows(h, &bm.dO32, ws + bp.off_dO, bp.Vw, (uint64_t)p.N, BH, 32, 3, "dO slices")) != FIPA_OK ||
+        (mst = encode_rows(h, &bm.Q32, w.Q, p.Kq, (uint64_t)p.N, BH, 32, 3, "Qhat slices")) != FIPA_OK)
       return mst;
     bm.ws = workspace;
     bm.dims = *dims;
@@ -610,7 +613,7 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
     if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
       return cuda_fail(h, "core launch", e);
   }
-  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, ctl, s,
+  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, bm.Q32, bm.dO32, ctl, s,
                                  rec ? +mark : nullptr, &mk)) != cudaSuccess)
     return cuda_fail(h, "backward launch", e);
   h->bwd_timed_call = rec;

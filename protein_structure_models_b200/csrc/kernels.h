@@ -117,7 +117,8 @@ struct BwdIO {
 typedef void (*StageMark)(void* ctx, int k);
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const DeviceCtl& ctl, cudaStream_t s,
+                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const CUtensorMap& tmQ32,
+                            const CUtensorMap& tmdO32, const DeviceCtl& ctl, cudaStream_t s,
                             StageMark mark = nullptr, void* mark_ctx = nullptr);
 
 // The IPA layer around the core (layer.cu), float32.
