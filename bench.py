@@ -45,6 +45,9 @@ import workloads  # noqa: E402
 METRIC = "fused IPA fwd query-key pairs/sec (B·H·N²/s), % of B200 BF16 tensor peak"
 UNIT = "pairs/s"
 DEFAULT_WORKLOAD = "3-16384"
+MATH = {"bf16": "fp16 tensor-core products, fp32 accumulate; bf16 inputs",
+        "f32": "fp16 tensor-core products of hi/lo splits (every float32 value as 2-3 fp16 parts), fp32 "
+               "accumulate, point distances in fp32 on the CUDA cores; float32 inputs"}
 
 
 def parse_args():
@@ -55,6 +58,8 @@ def parse_args():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
                     help="0, 1, 2, 4 or 3-<N> (length sweep, N in 512..16384)")
     ap.add_argument("--impl", choices=("fipa", "reference"), default="fipa")
+    ap.add_argument("--dtype", choices=("bf16", "f32"), default=None,
+                    help="input dtype of the workload (default: the workload's own)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--shard", choices=("auto", "replicas", "rows"), default="auto",
                     help="N > 1 GPUs: independent replicas (weak scaling) or the query rows of one "
@@ -702,7 +707,7 @@ def main_fipa(args, wl):
                                        (f"replicas x{world}" if r["mode"] == "replicas"
                                         else f"query-row shards x{world}"),
                                        "l2": "flushed (256 MB write) between timed steps",
-                                       "math": "fp16 tensor-core products, fp32 accumulate; bf16 inputs"}),
+                                       "math": MATH[wl.dtype]}),
         "valid_pairs_per_s": valid * mult / (r["step_ms"] / 1e3),
         "stage_ms": r["stage_ms"],
         "stage_check": r["stage_check"],
@@ -896,6 +901,8 @@ def main():
         main_sweep(args)
         return
     wl = workloads.workload(args.workload)
+    if args.dtype is not None:
+        wl = wl.with_(dtype=args.dtype)
     if args.impl == "reference":
         main_reference(args, wl)
     else:

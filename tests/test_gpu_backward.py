@@ -86,6 +86,23 @@ def test_backward_small_masks_and_empty_rows(handle):
     check_grads(handle, inp)
 
 
+def test_backward_masked_tiles_and_pair_mask(handle):
+    """Fully masked query and key tiles between valid ones (the forward's early
+    exit, the k side's zeroed rows) and a pair mask over a ragged last tile
+    (N = 300: the mask bits past N)."""
+    inp = _custom(23, N=384)
+    rng = np.random.default_rng(23)
+    m = rng.random((2, 384)) < 0.8
+    m[0, 128:256] = False
+    m[1, :128] = False
+    inp["mask"] = m
+    inp["pair_mask"] = rng.random((2, 384, 384)) < 0.7
+    check_grads(handle, inp)
+    inp = _custom(29, N=300, B=1)
+    inp["pair_mask"] = rng.random((1, 300, 300)) < 0.5
+    check_grads(handle, inp, seed=29)
+
+
 @pytest.mark.parametrize("N", [1, 129, 300])
 def test_backward_ragged_tiles(handle, N):
     inp = _custom(100 + N, N=N, B=1 if N == 300 else 2)

@@ -115,6 +115,24 @@ def test_masks_and_empty_rows(handles, dtype):
     check(handles, inp, dtype, want_attention=False)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_fully_masked_query_tiles(handles, dtype):
+    """A query tile without a valid residue leaves the core at entry, writing
+    only what an empty row gets (row statistics, lse -inf, zero local points,
+    the row flag): a masked middle tile and a masked first tile between valid
+    ones, with and without a pair mask."""
+    inp = _custom(dtype, 21, N=384)
+    rng = np.random.default_rng(21)
+    m = rng.random((2, 384)) < 0.8
+    m[0, 128:256] = False
+    m[1, :128] = False
+    inp["mask"] = m
+    check(handles, inp, dtype)
+    check(handles, inp, dtype, want_attention=False)
+    inp["pair_mask"] = rng.random((2, 384, 384)) < 0.7
+    check(handles, inp, dtype)
+
+
 def test_single_head_single_point(handles):
     inp = _custom("bf16", 11, N=64, H=1, P=1, Q=1, D=1, Dv=1, Cz=1, R=1, Cout=1)
     check(handles, inp, "bf16")
