@@ -1510,23 +1510,43 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
   }
 }
 
-// dWb[c, h] and d point_w_raw[h]: the chain CTAs' partial sums added in CTA
-// order; d raw = d g * 1/2 sigmoid(raw) sqrt(2/(27P)) (softplus' = sigmoid).
-__global__ void bwd_final_kernel(const BwdArgs a) {
+// dWb[c, h] and d point_w_raw[h]: the chain CTAs' partial sums, added in a
+// fixed order (deterministic): 32 outputs per CTA, one per lane; warp g of the
+// 8 sums the partials k = g, g + 8, ... in four interleaved accumulators (the
+// loads in flight together), and lane e of warp 0 adds the 8 warps' sums in
+// order.  d raw = d g * 1/2 sigmoid(raw) sqrt(2/(27P)) (softplus' = sigmoid).
+constexpr int kFinalOut = 32;
+__global__ void __launch_bounds__(256) bwd_final_kernel(const BwdArgs a) {
+  __shared__ float red[8][kFinalOut + 1];
   const Plan& p = a.p;
-  const int CH = p.Cz * p.H;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e < CH) {
+  const int CH = p.Cz * p.H, nout = CH + p.H, nk = a.bp.nchain;
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int e = blockIdx.x * kFinalOut + lane;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  if (e < nout) {
+    const float* src = e < CH ? a.wbpart + e : a.gpart + (e - CH);
+    const size_t stride = e < CH ? (size_t)CH : (size_t)p.H;
+    for (int k = grp; k < nk; k += 32) {
+      acc0 += src[(size_t)k * stride];
+      if (k + 8 < nk) acc1 += src[(size_t)(k + 8) * stride];
+      if (k + 16 < nk) acc2 += src[(size_t)(k + 16) * stride];
+      if (k + 24 < nk) acc3 += src[(size_t)(k + 24) * stride];
+    }
+  }
+  red[grp][lane] = (acc0 + acc1) + (acc2 + acc3);
+  __syncthreads();
+  if (grp == 0 && e < nout) {
     float s = 0.f;
-    for (int k = 0; k < a.bp.nchain; ++k) s += a.wbpart[(size_t)k * CH + e];
-    a.g.Wb[e] = s;
-  } else if (e < CH + p.H) {
-    const int h = e - CH;
-    float s = 0.f;
-    for (int k = 0; k < a.bp.nchain; ++k) s += a.gpart[(size_t)k * p.H + h];
-    const float raw = bwd_raw(a, h);
-    const float sig = 1.f / (1.f + expf(-raw));
-    a.g.raw[h] = s * 0.5f * sig * sqrtf(2.f / (27.f * (float)p.P));
+#pragma unroll
+    for (int g = 0; g < 8; ++g) s += red[g][lane];
+    if (e < CH) {
+      a.g.Wb[e] = s;
+    } else {
+      const int h = e - CH;
+      const float raw = bwd_raw(a, h);
+      const float sig = 1.f / (1.f + expf(-raw));
+      a.g.raw[h] = s * 0.5f * sig * sqrtf(2.f / (27.f * (float)p.P));
+    }
   }
 }
 
@@ -1609,7 +1629,7 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   bwd_dw_reduce_kernel<<<cdiv((p.F + 1) * p.Cout, 256), 256, 0, s>>>(a.dwpart, io.g.w_out, io.g.b_out, p.F, bp.Fp,
                                                                       p.Cout, bp.dw_ks);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  bwd_final_kernel<<<cdiv(p.Cz * p.H + p.H, 256), 256, 0, s>>>(a);
+  bwd_final_kernel<<<cdiv(p.Cz * p.H + p.H, kFinalOut), 256, 0, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage(5);
   return cudaSuccess;
