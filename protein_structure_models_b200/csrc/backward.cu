@@ -44,7 +44,8 @@ struct BwdArgs {
   const uint8_t* rowflag;
   float* osave;
   float* dfeat;
-  float* featp;
+  __nv_bfloat16* fhi;               // feature rows [F | 1 | 0..] as bfloat16 hi / lo (the dw_out operand)
+  __nv_bfloat16* flo;
   __half* dO;
   float4* dvec;
   float* rloc;
@@ -66,98 +67,9 @@ __device__ __forceinline__ float ldi(const void* p, size_t i, int f32) {
   return f32 ? static_cast<const float*>(p)[i] : __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]);
 }
 
-// ------------------------------------------------------------------ SIMT GEMMs
-// dfeat[m, n] = sum_k dupd[m, k] w[n, k]: the cotangent of the features,
-// d_update @ w_out^T (M = B*N rows, N = F features, K = Cout).
-__global__ void __launch_bounds__(256) bwd_dfeat_kernel(const float* __restrict__ A, const void* __restrict__ W,
-                                                        int w_f32, float* __restrict__ C, int M, int N, int K) {
-  __shared__ __align__(16) float As[32][68];
-  __shared__ __align__(16) float Ws[32][68];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < K; k0 += 32) {
-    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
-      const int r = e >> 5, kk = e & 31, k = k0 + kk;
-      As[kk][r] = (m0 + r < M && k < K) ? A[(size_t)(m0 + r) * K + k] : 0.f;
-      Ws[kk][r] = (n0 + r < N && k < K) ? ldi(W, (size_t)(n0 + r) * K + k, w_f32) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 wv = *reinterpret_cast<const float4*>(&Ws[kk][tx * 4]);
-      const float aa[4] = {av.x, av.y, av.z, av.w}, ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(aa[i], ww[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= M) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = n0 + tx * 4 + j;
-      if (n < N) C[(size_t)m * N + n] = acc[i][j];
-    }
-  }
-}
-
-// part[z, f, c] = sum over rows i of split z of featp[i, f] dupd[i, c]: the
-// weight gradient features^T d_update, split over rows (deterministic: the
-// splits are added in order by bwd_dw_reduce_kernel).  Row F of featp is 1 on
-// rows with a non-empty neighbourhood, so part[., F, .] sums d_update there.
-__global__ void __launch_bounds__(256) bwd_dw_kernel(const float* __restrict__ featp, const float* __restrict__ dupd,
-                                                     float* __restrict__ part, int M, int Fp, int Cout, int rps) {
-  __shared__ __align__(16) float As[32][68];
-  __shared__ __align__(16) float Bs[32][68];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const int f0 = blockIdx.y * 64, c0 = blockIdx.x * 64, z = blockIdx.z;
-  const int r0 = z * rps, r1 = min(M, r0 + rps);
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int i0 = r0; i0 < r1; i0 += 32) {
-    for (int e = threadIdx.x; e < 64 * 32; e += 256) {
-      const int kk = e >> 6, col = e & 63, i = i0 + kk;
-      As[kk][col] = (i < r1 && f0 + col < Fp) ? featp[(size_t)i * Fp + f0 + col] : 0.f;
-      Bs[kk][col] = (i < r1 && c0 + col < Cout) ? dupd[(size_t)i * Cout + c0 + col] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < 32; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
-      const float4 bv = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
-      const float aa[4] = {av.x, av.y, av.z, av.w}, bb[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(aa[i], bb[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int f = f0 + ty * 4 + i;
-    if (f >= Fp) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
-      if (c < Cout) part[((size_t)z * Fp + f) * Cout + c] = acc[i][j];
-    }
-  }
-}
-
+// ------------------------------------------------------------------ dw_out reduce
+// The dense products dfeat = d_update w_out^T and features^T d_update run on
+// the tensor cores (bgemm.cu); the latter's row splits are added here in order.
 // dw_out[f, c] = sum_z part[z, f, c] (f < F), db_out[c] = sum_z part[z, F, c].
 __global__ void bwd_dw_reduce_kernel(const float* __restrict__ part, float* __restrict__ dw, float* __restrict__ db,
                                      int F, int Fp, int Cout, int ks) {
@@ -179,6 +91,13 @@ __global__ void bwd_dw_reduce_kernel(const float* __restrict__ part, float* __re
 // D = fp16(dO) . O and sG = sum_q fp16(dG_q); the parts of the chain rule that
 // stay on this residue (local = R^T (G - t): dR += (G - t) (x) d local,
 // dt -= dG; dz1 += U d o_pair), and the fp32 feature row for dw_out.
+// Feature value v at flat index idx of the bfloat16 hi / lo feature rows.
+__device__ __forceinline__ void put_feat(const BwdArgs& a, size_t idx, float v) {
+  const __nv_bfloat16 hv = __float2bfloat16_rn(v);
+  a.fhi[idx] = hv;
+  a.flo[idx] = __float2bfloat16_rn(v - __bfloat162float(hv));
+}
+
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
   const Plan& p = a.p;
   const BwdPlan& bp = a.bp;
@@ -201,7 +120,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     }
     if (tid < 12) a.rloc[bi * 12 + tid] = 0.f;
     for (int e = tid; e < RCz; e += 256) a.dz1u[bi * RCz + e] = 0.f;
-    for (int e = tid; e < bp.Fp; e += 256) a.featp[bi * bp.Fp + e] = 0.f;
+    for (int e = tid; e < bp.Fp; e += 256) put_feat(a, bi * bp.Fp + e, 0.f);
     return;
   }
   for (int e = tid; e < F; e += 256) df[e] = a.dfeat[bi * F + e];
@@ -237,11 +156,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
 #pragma unroll
       for (int x = 0; x < 3; ++x) acc[3 * y + x] += gt[y] * dl[x];
     }
-    float* fr = a.featp + bi * bp.Fp;
-    fr[HDv + h * Q + q] = loc[0];
-    fr[HDv + HQ + h * Q + q] = loc[1];
-    fr[HDv + 2 * HQ + h * Q + q] = loc[2];
-    fr[HDv + 3 * HQ + h * Q + q] = len;
+    const size_t fr = bi * bp.Fp;
+    put_feat(a, fr + HDv + h * Q + q, loc[0]);
+    put_feat(a, fr + HDv + HQ + h * Q + q, loc[1]);
+    put_feat(a, fr + HDv + 2 * HQ + h * Q + q, loc[2]);
+    put_feat(a, fr + HDv + 3 * HQ + h * Q + q, len);
   }
 #pragma unroll
   for (int k = 0; k < 12; ++k) red[k * 256 + tid] = acc[k];
@@ -302,7 +221,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     if (lane == 0) a.dvec[(size_t)(b * H + h) * p.N + i] = make_float4(Dp, sx, sy, sz);
   }
   // dz1 from the pair aggregate, and the scalar / pair feature blocks
-  float* fr = a.featp + bi * bp.Fp;
+  const size_t fr = bi * bp.Fp;
   for (int rc = tid; rc < RCz; rc += 256) {
     const int cc = rc % Cz;
     float s = 0.f;
@@ -311,16 +230,16 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
   }
   for (int e = tid; e < HDv; e += 256) {
     const int h = e / Dv, d = e - h * Dv;
-    fr[e] = a.osave[(bi * H + h) * (size_t)bp.Osw + d];
+    put_feat(a, fr + e, a.osave[(bi * H + h) * (size_t)bp.Osw + d]);
   }
   for (int e = tid; e < H * Cz; e += 256) {
     const int h = e / Cz, c = e - h * Cz;
     const float* U = a.osave + (bi * H + h) * (size_t)bp.Osw + Dv + 3 * Q;
     float s = 0.f;
     for (int r = 0; r < p.R; ++r) s = fmaf(ldi(a.z1, bi * RCz + r * Cz + c, a.p.in_f32), U[r * Cz + c], s);
-    fr[pairblk + e] = s;
+    put_feat(a, fr + pairblk + e, s);
   }
-  for (int e = F + tid; e < bp.Fp; e += 256) fr[e] = e == F ? 1.f : 0.f;
+  for (int e = F + tid; e < bp.Fp; e += 256) put_feat(a, fr + e, e == F ? 1.f : 0.f);
 }
 
 // ------------------------------------------------------------------ shared pieces
@@ -1561,8 +1480,7 @@ size_t bwd_chain_smem(const Plan& p) {
 
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const CUtensorMap& tmQ32,
-                            const CUtensorMap& tmdO32, const DeviceCtl& ctl, cudaStream_t s,
+                            const CUtensorMap& tmZ, const BwdMaps& bm, const DeviceCtl& ctl, cudaStream_t s,
                             StageMark mark, void* mark_ctx) {
   auto stage = [&](int k) {
     if (mark != nullptr) mark(mark_ctx, k);
@@ -1578,7 +1496,8 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   uint8_t* ws = io.ws;
   a.osave = reinterpret_cast<float*>(ws + bp.off_osave);
   a.dfeat = reinterpret_cast<float*>(ws + bp.off_dfeat);
-  a.featp = reinterpret_cast<float*>(ws + bp.off_featp);
+  a.fhi = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_fhi);
+  a.flo = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_flo);
   a.dO = reinterpret_cast<__half*>(ws + bp.off_dO);
   a.dvec = reinterpret_cast<float4*>(ws + bp.off_dvec);
   a.rloc = reinterpret_cast<float*>(ws + bp.off_rloc);
@@ -1596,9 +1515,28 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   const int BN = p.B * p.N;
   cudaError_t e;
   stage(1);
-  bwd_dfeat_kernel<<<dim3(cdiv(p.F, 64), cdiv(BN, 64)), 256, 0, s>>>(
-      io.d_update, in.w_out, p.in_f32, a.dfeat, BN, p.F, p.Cout);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dfeat = d_update w_out^T: d_update and w_out as bfloat16 hi / lo rows of Coutp
+  // columns; w_out given in bfloat16 is exact in its hi part
+  __nv_bfloat16* duhi = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_duhi);
+  __nv_bfloat16* dulo = reinterpret_cast<__nv_bfloat16*>(ws + bp.off_dulo);
+  if ((e = launch_bsplit(io.d_update, 1, duhi, dulo, BN, p.Cout, bp.Coutp, s)) != cudaSuccess) return e;
+  if ((e = launch_bsplit(in.w_out, p.in_f32, reinterpret_cast<__nv_bfloat16*>(ws + bp.off_whi),
+                         reinterpret_cast<__nv_bfloat16*>(ws + bp.off_wlo), p.F, p.Cout, bp.Coutp, s)) != cudaSuccess)
+    return e;
+  {
+    BGemm g{};
+    g.A[0] = bm.duA[0]; g.A[1] = bm.duA[1]; g.B[0] = bm.w[0]; g.B[1] = bm.w[1];
+    g.a_mn = 0; g.b_mn = 0;
+    g.M = BN; g.N = p.F; g.K = bp.Coutp;
+    g.nparts = p.in_f32 ? 3 : 2;
+    g.pa[0] = 0; g.pb[0] = 0;      // d hi  w hi
+    g.pa[1] = 1; g.pb[1] = 0;      // d lo  w hi
+    g.pa[2] = 0; g.pb[2] = 1;      // d hi  w lo (float32 w_out)
+    g.splits = 1;
+    g.C = a.dfeat; g.ldc = p.F; g.zstride = 0;
+    g.status = ctl.status; g.timeout_ns = ctl.timeout_ns;
+    if ((e = launch_bgemm(g, s)) != cudaSuccess) return e;
+  }
   const size_t psm = bwd_prep_smem(p);
   if (psm > 48 * 1024) {
     if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm)) != cudaSuccess)
@@ -1608,11 +1546,11 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_q_kernel))) != cudaSuccess) return e;
   stage(2);
-  bwd_q_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.q_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, a);
+  bwd_q_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.q_smem, s>>>(tmQ, tmKH, tmVH, tmZ, *bm.dO, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_k_kernel))) != cudaSuccess) return e;
   stage(3);
-  bwd_k_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.k_smem, s>>>(tmQ, tmKH, tmVH, tmZ, tmdO, tmQ32, tmdO32, a);
+  bwd_k_kernel<<<dim3(p.nT, p.H, p.B), 256, bp.k_smem, s>>>(tmQ, tmKH, tmVH, tmZ, *bm.dO, *bm.Q32, *bm.dO32, a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   stage(4);
   const size_t csm = bwd_chain_smem(p);
@@ -1622,10 +1560,22 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
   }
   bwd_chain_kernel<<<bp.nchain, 256, csm, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int rps = cdiv(BN, bp.dw_ks);
-  bwd_dw_kernel<<<dim3(cdiv(p.Cout, 64), cdiv(bp.Fp, 64), bp.dw_ks), 256, 0, s>>>(a.featp, io.d_update, a.dwpart, BN,
-                                                                                  bp.Fp, p.Cout, rps);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    // [dw_out | db_out] partials = features^T d_update over row splits (the
+    // feature rows carry a 1 in column F, so row F of the result is db_out)
+    BGemm g{};
+    g.A[0] = bm.f[0]; g.A[1] = bm.f[1]; g.B[0] = bm.duB[0]; g.B[1] = bm.duB[1];
+    g.a_mn = 1; g.b_mn = 1;
+    g.M = bp.Fp; g.N = p.Cout; g.K = BN;
+    g.nparts = 3;
+    g.pa[0] = 0; g.pb[0] = 0;      // f hi  d hi
+    g.pa[1] = 0; g.pb[1] = 1;      // f hi  d lo
+    g.pa[2] = 1; g.pb[2] = 0;      // f lo  d hi
+    g.splits = bp.dw_ks;
+    g.C = a.dwpart; g.ldc = p.Cout; g.zstride = (size_t)bp.Fp * p.Cout;
+    g.status = ctl.status; g.timeout_ns = ctl.timeout_ns;
+    if ((e = launch_bgemm(g, s)) != cudaSuccess) return e;
+  }
   bwd_dw_reduce_kernel<<<cdiv((p.F + 1) * p.Cout, 256), 256, 0, s>>>(a.dwpart, io.g.w_out, io.g.b_out, p.F, bp.Fp,
                                                                       p.Cout, bp.dw_ks);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

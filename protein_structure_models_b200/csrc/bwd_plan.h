@@ -3,7 +3,7 @@
 //
 // The backward recomputes the forward (lift and fused core, the core also
 // saving the normalised aggregates O of every row), then:
-//   dfeat  = d_update @ w_out^T                                (SIMT GEMM)
+//   dfeat  = d_update @ w_out^T              (tcgen05, bfloat16 hi/lo parts)
 //   prep   per residue: dO = [d o_scalar | dG | dG | dU], D = dO . O, the
 //          frame and pair-value parts of the chain rule, fp32 features
 //   q-side per (query tile, head): S and dP recomputed on tcgen05, dS =
@@ -12,7 +12,7 @@
 //          dVhat = P^T dO and dz2 = dS^T u + P^T dU in tensor memory
 //   chain  per residue: points through the frames, z1 / z2 / Wb / point
 //          weights, deterministic partial sums
-//   dw_out = features^T d_update, db_out                        (SIMT GEMM)
+//   dw_out = features^T d_update, db_out     (tcgen05, bfloat16 hi/lo parts)
 #pragma once
 
 #include "plan.h"
@@ -33,12 +33,14 @@ struct BwdPlan {
   int tmDK, tmDV, tmDZ;   // k-side TMEM columns of the accumulators
   int Kr;         // q-side result row: [sum dS k (D) | X (3P) | rs | W (3) | E], padded to 4
   int Kk;         // k-side result row: [sum dS q/sqrt(3D) (D) | 2g Y (3P) | cs | V (3) | dv (Dv) | dg (3Q)], padded to 4
-  int Fp;         // fp32 feature row [F features | 1 | pad], padded to 64
+  int Fp;         // feature row [F features | 1 | pad], padded to 64 (bfloat16 hi and lo copies)
+  int Coutp;      // Cout padded to 64: row width of the bfloat16 copies of d_update and w_out
   int RCz;
   int chain_res;  // residues per chain CTA
   int nchain;     // chain CTAs
   int dw_ks;      // row splits of the dw_out GEMM
-  size_t off_lp, off_osave, off_dfeat, off_featp, off_dO, off_dvec, off_rloc, off_dz1u;
+  size_t off_lp, off_osave, off_dfeat, off_fhi, off_flo, off_duhi, off_dulo, off_whi, off_wlo, off_dO, off_dvec,
+      off_rloc, off_dz1u;
   size_t off_qres, off_du, off_kres, off_dz2h, off_dwpart, off_wbpart, off_gpart, total;
 };
 
@@ -88,12 +90,14 @@ static inline int make_bwd_plan(BwdPlan& b, const Plan& p, const char** why) {
   b.Kr = rup(p.D + 3 * p.P + 5, 4);
   b.Kk = rup(p.D + 3 * p.P + 4 + p.Dv + 3 * p.Q, 4);
   b.Fp = rup(p.F + 1, 64);
+  b.Coutp = rup(p.Cout, 64);
   b.chain_res = kChainRes;
   const int BN = p.B * p.N;
   b.nchain = cdiv(BN, kChainRes);
   {
-    const int tiles = cdiv(b.Fp, 64) * cdiv(p.Cout, 64);
-    int ks = cdiv(2 * 148, tiles);
+    // one wave of the dw_out GEMM's 128 x 256 tiles, split over 64-row chunks
+    const int tiles = cdiv(b.Fp, 128) * cdiv(p.Cout, 256);
+    int ks = cdiv(148, tiles);
     const int maxks = cdiv(BN, 64);
     if (ks > maxks) ks = maxks;
     if (ks < 1) ks = 1;
@@ -105,7 +109,12 @@ static inline int make_bwd_plan(BwdPlan& b, const Plan& p, const char** why) {
   b.off_lp = take(BHN * 3 * p.Q * 4);          // local points of the recompute (not an output)
   b.off_osave = take(BHN * b.Osw * 4);
   b.off_dfeat = take(BNs * p.F * 4);
-  b.off_featp = take(BNs * b.Fp * 4);
+  b.off_fhi = take(BNs * b.Fp * 2);
+  b.off_flo = take(BNs * b.Fp * 2);
+  b.off_duhi = take(BNs * b.Coutp * 2);
+  b.off_dulo = take(BNs * b.Coutp * 2);
+  b.off_whi = take((size_t)p.F * b.Coutp * 2);
+  b.off_wlo = take((size_t)p.F * b.Coutp * 2);
   b.off_dO = take(BHN * b.Vw * 2);
   b.off_dvec = take(BHN * 16);
   b.off_rloc = take(BNs * 12 * 4);

@@ -52,13 +52,14 @@ struct fipa_handle {
     int sig[5] = {0, 0, 0, 0, 0};   // layout widths the maps were encoded for
     CUtensorMap Q, KH, VH, Z, A, B;
   } maps;
-  // the backward's maps, cached the same way: dO with 128-row boxes, and Qhat
-  // and dO with 32-row boxes (the k side's slices of the pair columns)
+  // the backward's maps, cached the same way: dO with 128-row boxes, Qhat and
+  // dO with 32-row boxes (the k side's slices of the pair columns), and the
+  // bfloat16 hi / lo operands of its two dense products
   struct BwdMapCache {
     bool valid = false;
     const void* ws = nullptr;
     fipa_dims dims{};
-    CUtensorMap dO, Q32, dO32;
+    CUtensorMap dO, Q32, dO32, duA[2], duB[2], w[2], f[2];
   } bmaps;
 };
 
@@ -580,6 +581,17 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
         (mst = encode_rows(h, &bm.dO32, ws + bp.off_dO, bp.Vw, (uint64_t)p.N, BH, 32, 3, "dO slices")) != FIPA_OK ||
         (mst = encode_rows(h, &bm.Q32, w.Q, p.Kq, (uint64_t)p.N, BH, 32, 3, "Qhat slices")) != FIPA_OK)
       return mst;
+    const uint64_t BN = (uint64_t)p.B * p.N;
+    const size_t du_off[2] = {bp.off_duhi, bp.off_dulo}, w_off[2] = {bp.off_whi, bp.off_wlo},
+                 f_off[2] = {bp.off_fhi, bp.off_flo};
+    for (int k = 0; k < 2; ++k) {
+      if ((mst = encode_rows(h, &bm.duA[k], ws + du_off[k], bp.Coutp, BN, 1, 128, 2, "d_update parts")) != FIPA_OK ||
+          (mst = encode_rows(h, &bm.duB[k], ws + du_off[k], bp.Coutp, BN, 1, 64, 2, "d_update parts")) != FIPA_OK ||
+          (mst = encode_rows(h, &bm.w[k], ws + w_off[k], bp.Coutp, (uint64_t)p.F, 1, 256, 2, "w_out parts")) !=
+              FIPA_OK ||
+          (mst = encode_rows(h, &bm.f[k], ws + f_off[k], bp.Fp, BN, 1, 64, 2, "feature parts")) != FIPA_OK)
+        return mst;
+    }
     bm.ws = workspace;
     bm.dims = *dims;
     bm.valid = true;
@@ -613,7 +625,9 @@ static fipa_status backward_impl(fipa_handle* h, const void* q, const void* k, c
     if ((e = fipa::launch_core(p, in, w, out, mc.Q, mc.KH, mc.VH, mc.Z, ctl, s, osave)) != cudaSuccess)
       return cuda_fail(h, "core launch", e);
   }
-  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, bm.dO, bm.Q32, bm.dO32, ctl, s,
+  const fipa::BwdMaps maps{&bm.dO, &bm.Q32, &bm.dO32, {&bm.duA[0], &bm.duA[1]}, {&bm.duB[0], &bm.duB[1]},
+                           {&bm.w[0], &bm.w[1]}, {&bm.f[0], &bm.f[1]}};
+  if ((e = fipa::launch_backward(p, bp, in, w, io, mc.Q, mc.KH, mc.VH, mc.Z, maps, ctl, s,
                                  rec ? +mark : nullptr, &mk)) != cudaSuccess)
     return cuda_fail(h, "backward launch", e);
   h->bwd_timed_call = rec;

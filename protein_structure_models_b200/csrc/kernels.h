@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include <map>
@@ -115,10 +116,45 @@ struct BwdIO {
 // `mark(ctx, k)`, if given, is called before stage k = 1 (dfeat GEMM and prep),
 // 2 (q side), 3 (k side), 4 (chain and weight gradients) and after the last (5).
 typedef void (*StageMark)(void* ctx, int k);
+// TMA maps of the backward's own workspace regions (encoded on the host).
+struct BwdMaps {
+  const CUtensorMap* dO;       // dO rows, 128-row boxes
+  const CUtensorMap* Q32;      // Qhat, 32-row boxes (slices of the pair columns)
+  const CUtensorMap* dO32;     // dO, 32-row boxes
+  const CUtensorMap* duA[2];   // d_update hi / lo as the K-major A of dfeat (64 x 128 boxes)
+  const CUtensorMap* duB[2];   // d_update hi / lo as the MN-major B of dw_out (64 x 64 boxes)
+  const CUtensorMap* w[2];     // w_out hi / lo as the K-major B of dfeat (64 x 256 boxes)
+  const CUtensorMap* f[2];     // feature rows hi / lo as the MN-major A of dw_out (64 x 64 boxes)
+};
+
+// The backward's dense float32 products on the tensor cores (bgemm.cu):
+// C[M, N] (+ split z at C + z zstride) = sum over parts p of A_{pa[p]} B_{pb[p]}^T,
+// each float32 operand as bfloat16 hi (map 0) and lo (map 1) parts.  a_mn / b_mn:
+// 0 = K-major operand map (box 64 x 128 rows for A, 64 x 256 rows for B),
+// 1 = MN-major (rows = K, box 64 x 64).  Splits divide K in 64-wide chunks.
+struct BGemm {
+  const CUtensorMap* A[2];
+  const CUtensorMap* B[2];
+  int a_mn, b_mn;
+  int M, N, K;
+  int nparts;
+  int pa[3], pb[3];
+  int splits;
+  float* C;
+  int ldc;
+  size_t zstride;
+  int* status;
+  unsigned long long timeout_ns;
+};
+cudaError_t launch_bgemm(const BGemm& g, cudaStream_t s);
+int bgemm_tiles(int M, int N);
+// x [rows, cols] (float32, or bfloat16 when x_f32 = 0) -> bfloat16 hi, lo [rows, ldo]
+cudaError_t launch_bsplit(const void* x, int x_f32, __nv_bfloat16* hi, __nv_bfloat16* lo, int rows, int cols, int ldo,
+                          cudaStream_t s);
+
 cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, const Work& w, const BwdIO& io,
                             const CUtensorMap& tmQ, const CUtensorMap& tmKH, const CUtensorMap& tmVH,
-                            const CUtensorMap& tmZ, const CUtensorMap& tmdO, const CUtensorMap& tmQ32,
-                            const CUtensorMap& tmdO32, const DeviceCtl& ctl, cudaStream_t s,
+                            const CUtensorMap& tmZ, const BwdMaps& bm, const DeviceCtl& ctl, cudaStream_t s,
                             StageMark mark = nullptr, void* mark_ctx = nullptr);
 
 // The IPA layer around the core (layer.cu), float32.

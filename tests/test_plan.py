@@ -67,11 +67,11 @@ int main(int argc, char** argv) {
              b.q_smem, b.k_smem, b.q_nst, b.k_nst, b.nQr, b.nOc, b.k_nres);
       printf(", \"tmDS\": %d, \"tmDQ\": %d, \"tmDK\": %d, \"tmDV\": %d, \"tmDZ\": %d, \"Vw\": %d, \"Kr\": %d, \"Kk\": %d, \"Fp\": %d",
              b.tmDS, b.tmDQ, b.tmDK, b.tmDV, b.tmDZ, b.Vw, b.Kr, b.Kk, b.Fp);
-      const size_t bo[] = {b.off_lp, b.off_osave, b.off_dfeat, b.off_featp, b.off_dO, b.off_dvec, b.off_rloc,
-                           b.off_dz1u, b.off_qres, b.off_du, b.off_kres, b.off_dz2h, b.off_dwpart, b.off_wbpart,
-                           b.off_gpart, b.total};
+      const size_t bo[] = {b.off_lp, b.off_osave, b.off_dfeat, b.off_fhi, b.off_flo, b.off_duhi, b.off_dulo,
+                           b.off_whi, b.off_wlo, b.off_dO, b.off_dvec, b.off_rloc, b.off_dz1u, b.off_qres, b.off_du,
+                           b.off_kres, b.off_dz2h, b.off_dwpart, b.off_wbpart, b.off_gpart, b.total};
       printf(", \"offs\": [");
-      for (int i = 0; i < 16; ++i) printf("%s%zu", i ? ", " : "", bo[i]);
+      for (int i = 0; i < 21; ++i) printf("%s%zu", i ? ", " : "", bo[i]);
       printf("]");
     }
     printf("}");
