@@ -98,42 +98,55 @@ __device__ __forceinline__ void put_feat(const BwdArgs& a, size_t idx, float v) 
   a.flo[idx] = __float2bfloat16_rn(v - __bfloat162float(hv));
 }
 
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
+// WPR warps per residue (b, i): 1 (a CTA holds `wpc` residues; many
+// residues) or 8 (one residue per CTA; few residues, more threads each).  The
+// group's shared memory holds dG [H][3Q]; sums over a residue's items (the
+// frame terms, D) are per-thread partial sums added in a fixed order (warp
+// shuffle tree, then the warps in order).
+template <int WPR>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a, int wpc) {
   const Plan& p = a.p;
   const BwdPlan& bp = a.bp;
   extern __shared__ float psm[];
+  constexpr int T = 32 * WPR;                                 // threads per residue
   const int H = p.H, Dv = p.Dv, Q = p.Q, Cz = p.Cz, RCz = bp.RCz, F = p.F;
   const int HDv = H * Dv, HQ = H * Q, pairblk = HDv + 4 * HQ;
-  const size_t bi = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = WPR == 1 ? warp : 0;                        // residue slot in the CTA
+  const int gw = WPR == 1 ? 0 : warp;                         // warp within the residue
+  const int gt = gw * 32 + lane;                              // thread within the residue
+  const size_t bi = (size_t)blockIdx.x * wpc + grp;
+  if (bi >= (size_t)p.B * p.N) return;                       // whole groups only
   const int b = (int)(bi / p.N), i = (int)(bi - (size_t)b * p.N);
-  float* df = psm;                                   // [F]
-  float* sdG = df + rup(F, 4);                       // [H][3Q]
-  float* red = sdG + rup(H * 3 * Q, 4);              // [12][256]
-  float* Rt = red + 12 * 256;                        // R (9), t (3)
-  const int tid = threadIdx.x;
-  const bool live = a.rowflag[bi] != 0;
-  if (!live) {
-    for (int h = 0; h < H; ++h) {
+  float* sdG = psm + (size_t)grp * rup(H * 3 * Q, 4);        // [H][3Q]
+  float* red = psm + (size_t)(WPR == 1 ? wpc : 1) * rup(H * 3 * Q, 4);   // [WPR][12] (WPR > 1)
+  auto group_sync = [&]() {
+    if (WPR == 1) __syncwarp();
+    else __syncthreads();
+  };
+  const float* df = a.dfeat + bi * F;
+  const size_t fr = bi * bp.Fp;
+  if (a.rowflag[bi] == 0) {                                   // uniform over the group
+    for (int h = gw; h < H; h += WPR) {
       uint4* drow = reinterpret_cast<uint4*>(a.dO + ((size_t)(b * H + h) * p.N + i) * bp.Vw);
-      for (int c = tid; c < bp.Vw / 8; c += 256) drow[c] = make_uint4(0u, 0u, 0u, 0u);
-      if (tid == 0) a.dvec[(size_t)(b * H + h) * p.N + i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = lane; c < bp.Vw / 8; c += 32) drow[c] = make_uint4(0u, 0u, 0u, 0u);
+      if (lane == 0) a.dvec[(size_t)(b * H + h) * p.N + i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (tid < 12) a.rloc[bi * 12 + tid] = 0.f;
-    for (int e = tid; e < RCz; e += 256) a.dz1u[bi * RCz + e] = 0.f;
-    for (int e = tid; e < bp.Fp; e += 256) put_feat(a, bi * bp.Fp + e, 0.f);
+    if (gt < 12) a.rloc[bi * 12 + gt] = 0.f;
+    for (int e = gt; e < RCz; e += T) a.dz1u[bi * RCz + e] = 0.f;
+    for (int e = gt; e < bp.Fp; e += T) put_feat(a, fr + e, 0.f);
     return;
   }
-  for (int e = tid; e < F; e += 256) df[e] = a.dfeat[bi * F + e];
-  if (tid < 9) Rt[tid] = ldi(a.rot, bi * 9 + tid, a.p.in_f32);
-  else if (tid < 12) Rt[tid] = ldi(a.trans, bi * 3 + tid - 9, a.p.in_f32);
-  __syncthreads();
-  const float* R = Rt;
-  const float* t = Rt + 9;
-  // points: (h, q) items
+  float R[9], t[3];
+#pragma unroll
+  for (int e = 0; e < 9; ++e) R[e] = ldi(a.rot, bi * 9 + e, a.p.in_f32);
+#pragma unroll
+  for (int e = 0; e < 3; ++e) t[e] = ldi(a.trans, bi * 3 + e, a.p.in_f32);
+  // points: (h, q) items over the lanes
   float acc[12];
 #pragma unroll
   for (int k = 0; k < 12; ++k) acc[k] = 0.f;
-  for (int it = tid; it < HQ; it += 256) {
+  for (int it = gt; it < HQ; it += T) {
     const int h = it / Q, q = it - h * Q;
     const float* G = a.osave + (bi * H + h) * (size_t)bp.Osw + Dv + 3 * q;
     const float gt[3] = {G[0] - t[0], G[1] - t[1], G[2] - t[2]};
@@ -141,11 +154,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
 #pragma unroll
     for (int x = 0; x < 3; ++x) loc[x] = R[x] * gt[0] + R[3 + x] * gt[1] + R[6 + x] * gt[2];
     const float len = sqrtf(loc[0] * loc[0] + loc[1] * loc[1] + loc[2] * loc[2] + a.eps);
-    const float dlen = df[HDv + 3 * HQ + h * Q + q];
+    const float dlen = __ldg(df + HDv + 3 * HQ + h * Q + q);
     float dl[3];
 #pragma unroll
     for (int x = 0; x < 3; ++x) {
-      dl[x] = df[HDv + x * HQ + h * Q + q] + dlen * loc[x] / len;
+      dl[x] = __ldg(df + HDv + x * HQ + h * Q + q) + dlen * loc[x] / len;
       if (a.d_local != nullptr) dl[x] += a.d_local[((bi * H + h) * Q + q) * 3 + x];
     }
 #pragma unroll
@@ -156,25 +169,32 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
 #pragma unroll
       for (int x = 0; x < 3; ++x) acc[3 * y + x] += gt[y] * dl[x];
     }
-    const size_t fr = bi * bp.Fp;
     put_feat(a, fr + HDv + h * Q + q, loc[0]);
     put_feat(a, fr + HDv + HQ + h * Q + q, loc[1]);
     put_feat(a, fr + HDv + 2 * HQ + h * Q + q, loc[2]);
     put_feat(a, fr + HDv + 3 * HQ + h * Q + q, len);
   }
+  float mine = 0.f;
 #pragma unroll
-  for (int k = 0; k < 12; ++k) red[k * 256 + tid] = acc[k];
-  __syncthreads();
-  for (int s = 128; s > 0; s >>= 1) {
-    if (tid < s)
+  for (int k = 0; k < 12; ++k) {
+    float v = acc[k];
 #pragma unroll
-      for (int k = 0; k < 12; ++k) red[k * 256 + tid] += red[k * 256 + tid + s];
-    __syncthreads();
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == k) mine = v;
   }
-  if (tid < 12) a.rloc[bi * 12 + tid] = red[tid * 256];
-  // dO rows, D and sG: one warp per head
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int h = warp; h < H; h += 8) {
+  if (WPR == 1) {
+    if (lane < 12) a.rloc[bi * 12 + lane] = mine;
+  } else {
+    if (lane < 12) red[gw * 12 + lane] = mine;
+  }
+  group_sync();                                               // dG rows and warp sums visible
+  if (WPR > 1 && gt < 12) {
+    float v = 0.f;
+    for (int w = 0; w < WPR; ++w) v += red[w * 12 + gt];
+    a.rloc[bi * 12 + gt] = v;
+  }
+  // dO rows, D and sG: heads over the group's warps
+  for (int h = gw; h < H; h += WPR) {
     const float* Oh = a.osave + (bi * H + h) * (size_t)bp.Osw;
     uint4* drow = reinterpret_cast<uint4*>(a.dO + ((size_t)(b * H + h) * p.N + i) * bp.Vw);
     float Dp = 0.f;
@@ -188,7 +208,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
           const int c = c8 * 8 + e2 * 2 + u;
           float x = 0.f, o = 0.f;
           if (c < Dv) {
-            x = df[h * Dv + c];
+            x = __ldg(df + h * Dv + c);
             o = Oh[c];
           } else if (c >= p.Dv8 && c < p.Dv8 + 3 * Q) {
             x = sdG[h * 3 * Q + c - p.Dv8];
@@ -197,7 +217,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
             x = sdG[h * 3 * Q + c - p.Dv8 - p.Q38];       // second copy: meets g' lo, not part of D
           } else if (c >= p.VHp && c < p.VHp + RCz) {
             const int rc = c - p.VHp, cc = rc % Cz;
-            x = ldi(a.z1, bi * RCz + rc, a.p.in_f32) * df[pairblk + h * Cz + cc];
+            x = ldi(a.z1, bi * RCz + rc, a.p.in_f32) * __ldg(df + pairblk + h * Cz + cc);
             o = Oh[Dv + 3 * Q + rc];
           }
           xv[u] = x;
@@ -221,25 +241,25 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
     if (lane == 0) a.dvec[(size_t)(b * H + h) * p.N + i] = make_float4(Dp, sx, sy, sz);
   }
   // dz1 from the pair aggregate, and the scalar / pair feature blocks
-  const size_t fr = bi * bp.Fp;
-  for (int rc = tid; rc < RCz; rc += 256) {
+  for (int rc = gt; rc < RCz; rc += T) {
     const int cc = rc % Cz;
     float s = 0.f;
-    for (int h = 0; h < H; ++h) s = fmaf(a.osave[(bi * H + h) * (size_t)bp.Osw + Dv + 3 * Q + rc], df[pairblk + h * Cz + cc], s);
+    for (int h = 0; h < H; ++h)
+      s = fmaf(a.osave[(bi * H + h) * (size_t)bp.Osw + Dv + 3 * Q + rc], __ldg(df + pairblk + h * Cz + cc), s);
     a.dz1u[bi * RCz + rc] = s;
   }
-  for (int e = tid; e < HDv; e += 256) {
+  for (int e = gt; e < HDv; e += T) {
     const int h = e / Dv, d = e - h * Dv;
     put_feat(a, fr + e, a.osave[(bi * H + h) * (size_t)bp.Osw + d]);
   }
-  for (int e = tid; e < H * Cz; e += 256) {
+  for (int e = gt; e < H * Cz; e += T) {
     const int h = e / Cz, c = e - h * Cz;
     const float* U = a.osave + (bi * H + h) * (size_t)bp.Osw + Dv + 3 * Q;
     float s = 0.f;
     for (int r = 0; r < p.R; ++r) s = fmaf(ldi(a.z1, bi * RCz + r * Cz + c, a.p.in_f32), U[r * Cz + c], s);
     put_feat(a, fr + pairblk + e, s);
   }
-  for (int e = F + tid; e < bp.Fp; e += 256) put_feat(a, fr + e, e == F ? 1.f : 0.f);
+  for (int e = F + gt; e < bp.Fp; e += T) put_feat(a, fr + e, e == F ? 1.f : 0.f);
 }
 
 // ------------------------------------------------------------------ shared pieces
@@ -1416,8 +1436,10 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
     a.g.z1[(size_t)bi * RCz + rc] = s1;
     a.g.z2[(size_t)bi * RCz + rc] = s2;
   }
+  // dWb partials: consecutive threads take consecutive channels c (coalesced
+  // du and z1 rows); the result lands at [c][h]
   for (int e = tid; e < Cz * H; e += blockDim.x) {
-    const int c = e / H, h = e - c * H;
+    const int h = e / Cz, c = e - h * Cz;
     float s = 0.f;
     for (int r = 0; r < nres; ++r) {
       const int bi = bi0 + r, b = bi / N, i = bi - b * N;
@@ -1425,7 +1447,7 @@ __global__ void __launch_bounds__(256) bwd_chain_kernel(const BwdArgs a) {
       for (int rr = 0; rr < p.R; ++rr)
         s = fmaf(a.du[idx * RCz + rr * Cz + c], ldi(a.z1, (size_t)bi * RCz + rr * Cz + c, a.p.in_f32), s);
     }
-    a.wbpart[(size_t)blockIdx.x * Cz * H + e] = s * kInvSqrt3;
+    a.wbpart[(size_t)blockIdx.x * Cz * H + (size_t)c * H + h] = s * kInvSqrt3;
   }
 }
 
@@ -1471,8 +1493,19 @@ __global__ void __launch_bounds__(256) bwd_final_kernel(const BwdArgs a) {
 
 }  // namespace
 
+// The prep's form: one CTA of 8 warps per residue while the residues are
+// fewer than kPrepWarpMin (more threads per residue), else one warp per residue
+// and up to 8 residues per CTA (each warp's dG rows within 48 KB).
+constexpr int kPrepWarpMin = 8192;
+bool bwd_prep_cta(const Plan& p) { return p.B * p.N < kPrepWarpMin; }
+int bwd_prep_wpc(const Plan& p) {
+  if (bwd_prep_cta(p)) return 1;
+  const size_t per = (size_t)rup(p.H * 3 * p.Q, 4) * 4;
+  const size_t w = per > 0 ? 49152 / per : 8;
+  return w >= 8 ? 8 : (w < 1 ? 1 : (int)w);
+}
 size_t bwd_prep_smem(const Plan& p) {
-  return ((size_t)rup(p.F, 4) + rup(p.H * 3 * p.Q, 4) + 12 * 256 + 16) * 4;
+  return ((size_t)bwd_prep_wpc(p) * rup(p.H * 3 * p.Q, 4) + (bwd_prep_cta(p) ? 8 * 12 : 0)) * 4;
 }
 size_t bwd_chain_smem(const Plan& p) {
   return ((size_t)kChainRes * p.H * 13 + kChainRes * 16) * 4;
@@ -1537,12 +1570,17 @@ cudaError_t launch_backward(const Plan& p, const BwdPlan& bp, const Inputs& in, 
     g.status = ctl.status; g.timeout_ns = ctl.timeout_ns;
     if ((e = launch_bgemm(g, s)) != cudaSuccess) return e;
   }
+  const int wpc = bwd_prep_wpc(p);
   const size_t psm = bwd_prep_smem(p);
-  if (psm > 48 * 1024) {
-    if ((e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm)) != cudaSuccess)
+  if (bwd_prep_cta(p)) {
+    if (psm > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(bwd_prep_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm)) !=
+            cudaSuccess)
       return e;
+    bwd_prep_kernel<8><<<BN, 256, psm, s>>>(a, 1);
+  } else {
+    bwd_prep_kernel<1><<<cdiv(BN, wpc), 32 * wpc, psm, s>>>(a, wpc);
   }
-  bwd_prep_kernel<<<BN, 256, psm, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if ((e = allow_max_smem(reinterpret_cast<const void*>(bwd_q_kernel))) != cudaSuccess) return e;
   stage(2);
