@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--impl", choices=("fipa", "reference"), default="fipa")
     ap.add_argument("--dtype", choices=("bf16", "f32"), default=None,
                     help="input dtype of the workload (default: the workload's own)")
+    ap.add_argument("--n", type=int, default=None,
+                    help="residues per sample (default: the workload's own N); the other widths stay")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--shard", choices=("auto", "replicas", "rows"), default="auto",
                     help="N > 1 GPUs: independent replicas (weak scaling) or the query rows of one "
@@ -903,6 +905,8 @@ def main():
     wl = workloads.workload(args.workload)
     if args.dtype is not None:
         wl = wl.with_(dtype=args.dtype)
+    if args.n is not None:
+        wl = wl.with_(N=args.n, name=f"{wl.name}-N{args.n}")
     if args.impl == "reference":
         main_reference(args, wl)
     else:
