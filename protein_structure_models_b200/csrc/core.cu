@@ -747,19 +747,28 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const float* kpb = kpbuf + kb * kTile * P3;
         float aq[3 * kMaxPSimt];
         for (int x = 0; x < P3; ++x) aq[x] = in_range ? a.QP[((size_t)bh * N + i) * P3 + x] : 0.f;
+        // per group of 32 keys: one pass over the coordinates with 32 accumulators
+        // in registers (each key's sum still runs over x in order); a pass per
+        // key instead indexed aq and dd at run time, i.e. from local memory,
+        // and made this loop the float32 core's bound (3.6x slower at N = 4096)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const float dd[3] = {oqs.x - okg[t].x, oqs.y - okg[t].y, oqs.z - okg[t].z};
+          float d2[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float* kj = kpb + (t * 32 + e) * P3;
-            float d2 = 0.f;
-            for (int x = 0; x < P3; ++x) {
-              const float d = (aq[x] + dd[x % 3]) - kj[x];
-              d2 = fmaf(d, d, d2);
+          for (int e = 0; e < 32; ++e) d2[e] = 0.f;
+          const float* kt0 = kpb + t * 32 * P3;
+          for (int x = 0; x < P3; ++x) {
+            const int c = x % 3;
+            const float ax = aq[x] + (c == 0 ? dd[0] : (c == 1 ? dd[1] : dd[2]));
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float d = ax - kt0[e * P3 + x];
+              d2[e] = fmaf(d, d, d2[e]);
             }
-            sv[t][e] = __float_as_uint(__uint_as_float(sv[t][e]) - g * d2);
           }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) sv[t][e] = __float_as_uint(__uint_as_float(sv[t][e]) - g * d2[e]);
         }
       }
       mbar_arrive(&kt_empty[kb]);
