@@ -250,10 +250,12 @@ fipa_status fipa_backward_workspace_size(const fipa_handle* h, const fipa_dims* 
  * also keeps the normalised aggregates of every row) inside the workspace, so
  * it needs no state from an earlier fipa_forward.  Rows with an empty
  * neighbourhood have constant (zero) outputs and pass no gradient back.
- * Every product runs on fp16 tensor-core operands with fp32 accumulation, for
- * bfloat16 and float32 inputs alike (float32 inputs are recomputed in the
- * bfloat16 lifted layout); the gradients' normwise error is of the order of
- * 1e-3.  Allocates nothing, does not synchronise; kernels run on `stream`.
+ * The attention products run on fp16 tensor-core operands with fp32
+ * accumulation, for bfloat16 and float32 inputs alike (float32 inputs are
+ * recomputed in the bfloat16 lifted layout); the two dense products of the
+ * output projection (d_update w_out^T and features^T d_update) take every
+ * float32 operand as a bfloat16 hi + lo pair (about 2^-17 relative).  The
+ * gradients' normwise error is of the order of 1e-3.  Allocates nothing, does not synchronise; kernels run on `stream`.
  * Deterministic: every sum is taken in a fixed order. */
 fipa_status fipa_backward(fipa_handle* h,
                           const void* q, const void* k, const void* v,
