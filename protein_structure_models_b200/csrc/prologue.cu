@@ -20,23 +20,6 @@ namespace {
 
 constexpr int kLiftThreads = 256;
 
-__device__ __forceinline__ __half hi_half(float x) { return __float2half_rn(x); }
-__device__ __forceinline__ __half lo_half(float x) {
-  return __float2half_rn(x - __half2float(__float2half_rn(x)));
-}
-__device__ __forceinline__ uint32_t pack2(float a, float b, bool lo) {
-  const __half x = lo ? lo_half(a) : hi_half(a), y = lo ? lo_half(b) : hi_half(b);
-  return (uint32_t)__half_as_ushort(x) | ((uint32_t)__half_as_ushort(y) << 16);
-}
-__device__ __forceinline__ void store8(__half* dst, const float (&v)[8], bool lo) {
-  uint4 u;
-  u.x = pack2(v[0], v[1], lo);
-  u.y = pack2(v[2], v[3], lo);
-  u.z = pack2(v[4], v[5], lo);
-  u.w = pack2(v[6], v[7], lo);
-  *reinterpret_cast<uint4*>(dst) = u;
-}
-
 struct PrologueArgs {
   Plan p;
   Inputs in;
