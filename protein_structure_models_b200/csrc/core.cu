@@ -913,9 +913,25 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   // per-row state for the warps that did not run the softmax (the key-term
   // buffer is free now); the z1 copies of the softmax threads complete first
   float2* rowinfo = reinterpret_cast<float2*>(tail + kKtBuf);
+  // float32 inputs: the P.V product's own sum of P (the value column of ones),
+  // which normalises O: the tensor cores' fp32 accumulation of the aggregates
+  // then shares its rounding with the divisor, instead of drifting from the
+  // softmax's CUDA-core sum as the number of keys grows
+  float* rowlsum = reinterpret_cast<float*>(tail + kKtBuf + kTile * 8);
   if (warp >= 4) {
     cp_async_wait_all();
     rowinfo[(warp - 4) * 32 + lane] = make_float2(rowL, (row_ok && nkt > 0) ? 1.f : 0.f);
+    if (SPLIT && p.ones_col >= 0) {
+      float lt = 0.f;
+      const bool aborted = __any_sync(0xffffffffu, *abort_flag != 0);
+      if (nkt > 0 && !aborted) {                               // uniform over the warp
+        uint32_t o[32];
+        tmem_ld32(tmem + ((uint32_t)((warp - 4) * 32) << 16) + (uint32_t)(p.tmemO + (p.ones_col & ~31)), o);
+        tmem_ld_wait();
+        lt = __uint_as_float(o[p.ones_col & 31]);
+      }
+      rowlsum[(warp - 4) * 32 + lane] = lt;
+    }
   }
   __syncthreads();
   if (*abort_flag == 0) {
@@ -928,6 +944,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t trow = tmem + ((uint32_t)(wq * 32) << 16);
     const float2 ri = rowinfo[r];
     const float inv = ri.x > 0.f ? 1.f / ri.x : 0.f;
+    float inv_o = inv;                                        // divisor of the P.V aggregates
+    if (SPLIT && p.ones_col >= 0) {
+      const float lt = rowlsum[r];
+      inv_o = lt > 0.f ? 1.f / lt : inv;
+    }
     const bool live = ri.y != 0.f;
     const bool empty = !(ri.x > 0.f) || !live;
     const size_t bi = (size_t)b * N + (in_range ? i : 0);
@@ -942,7 +963,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv;
+          for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv_o;
         }
       }
       ttr.ev(45);
@@ -1010,11 +1031,11 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
               }
             }
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv, acc[e]);
+            for (int e = 0; e < 32; ++e) acc[e] = fmaf(zv[e], __uint_as_float(o[e]) * inv_o, acc[e]);
             if (SAVE) {
               float* us = a.osave + (bi * p.H + h) * (size_t)(p.Dv + 3 * p.Q + RCz) + p.Dv + 3 * p.Q + rr * Cz + c0;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) us[e] = __uint_as_float(o[e]) * inv;
+              for (int e = 0; e < 32; ++e) us[e] = __uint_as_float(o[e]) * inv_o;
             }
           }
         }

@@ -92,6 +92,7 @@ struct Plan {
   int geo_simt;       // 1: squared distance in fp32 on the CUDA cores (f32 inputs)
   int Kq, nQc;        // Qhat row width and chunks
   int VHc, VHp, nVH;  // value head-part columns, padded, chunks
+  int ones_col;       // float32 inputs: value column holding 1 (the P.V product's own sum of P), or -1
   int ZVc, nZV;       // pair columns used by the value product, chunks
   int Ocols;          // VHp + nZV * 64: fp32 accumulator columns per row
   int Pcols;          // TMEM columns holding P (64, or 128 for hi+lo)
@@ -174,6 +175,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   p.nQc = p.Kq / kChunk;
   p.VHc = p.nsv * p.Dv8 + 2 * p.Q38;
   p.VHp = rup(p.VHc, kChunk);
+  p.ones_col = (f32 && p.VHp > p.VHc) ? p.VHc : -1;
   p.nVH = p.VHp / kChunk;
   p.ZVc = p.nzv * p.RC8;
   p.nZV = cdiv(p.ZVc, kChunk);

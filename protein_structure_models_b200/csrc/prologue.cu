@@ -32,7 +32,7 @@ struct PrologueArgs {
 // holds, for each chunk position of each row type, which source it reads, at
 // which offset, and whether it stores the hi or the lo half; the write loop
 // then does no index arithmetic beyond one table load per chunk.
-enum : uint32_t { kSrcZero = 0, kSrcScalar = 1, kSrcPoint = 2, kSrcPair = 3, kSrcZ2 = 4 };
+enum : uint32_t { kSrcZero = 0, kSrcScalar = 1, kSrcPoint = 2, kSrcPair = 3, kSrcZ2 = 4, kSrcOne = 5 };
 enum : int { kRowQ = 0, kRowK = 1, kRowV = 2, kRowZ = 3 };
 
 __device__ __forceinline__ uint32_t make_desc(uint32_t src, int off, int woff, bool lo) {
@@ -58,6 +58,8 @@ __device__ uint32_t chunk_desc(const Plan& p, int rt, int col) {
       const int seg = (col - sv) / p.Q38;
       return make_desc(kSrcPoint, 2 * p.P38 + (col - sv - seg * p.Q38), 0, seg == 1);
     }
+    // float32 inputs: a column of ones (its own chunk; VHc is a multiple of 8)
+    if (col == p.ones_col) return make_desc(kSrcOne, 0, 0, false);
     return make_desc(kSrcZero, 0, 0, false);
   }
   // query (rt 0) and key (rt 1) head parts: the lo copy is segment 2 on the
@@ -166,6 +168,9 @@ __device__ __forceinline__ void chunk_values(uint32_t d, bool valid, const float
     lds8(prow + off, v);
 #pragma unroll
     for (int t = 0; t < 8; ++t) v[t] = ptscale * v[t];
+  } else if (src == kSrcOne) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) v[t] = t == 0 ? 1.f : 0.f;
   } else if (src == kSrcPair) {
     float w[8];
     lds8(z1row + off, v);

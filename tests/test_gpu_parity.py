@@ -48,6 +48,17 @@ def test_workload0_tiny_f32(handles):
     check(handles, inp, "f32")
 
 
+def test_workload0_float32_long_chain(handles):
+    """The float32 path on a long chain (N = 2048: 16 key tiles per query tile,
+    the exact point term over every key group, the aggregates normalised by
+    the tensor cores' own sum of P), on sampled rows."""
+    n = 2048
+    inp = workloads.make_inputs(workloads.workload(0).with_(N=n))
+    rng = np.random.default_rng(40)
+    rows = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.choice(n, 60, replace=False)]))
+    check(handles, inp, "f32", rows=rows, want_attention=False)
+
+
 def test_workload1_protein_batch(handles):
     inp = workloads.make_inputs(workloads.workload(1))
     check(handles, inp, "bf16")
