@@ -257,6 +257,17 @@ struct EpiLayout {
 __device__ __forceinline__ EpiLayout epi_layout(const Plan& p, const void* z1) {
   EpiLayout e;
   const uint32_t ring_end = (uint32_t)(p.nQres + (p.vbuf ? p.nVB : 0) + p.nst) * kChunkBytes;
+  if (p.oacc_T > 0) {
+    // float32 inputs with O in segments: the rows are staged in place in the
+    // fp32 accumulator (the tail), all columns, and z1 may use the Qhat region
+    e.fast_pair = false;
+    e.staged = p.Ocols;
+    e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.in_f32 ? 4 : 2));
+    e.z1_stride = e.z1_row_bytes + 16;
+    e.z1_smem = false;
+    e.o_off = ring_end + (uint32_t)p.oacc_off;
+    return e;
+  }
   e.fast_pair = (p.Cz % 32) == 0 && (reinterpret_cast<uintptr_t>(z1) & 15) == 0;
   e.staged = e.fast_pair ? p.VHp : p.Ocols;
   e.z1_row_bytes = (uint32_t)(p.R * p.Cz * (p.in_f32 ? 4 : 2));
@@ -603,7 +614,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t bd = desc_mnmajor_sw128(b0 + kk * 2048, kChunkBytes);
-            mma_ts(dcol, tmem + kTmemP + kk * 8, bd, idO, (s > 0 || kk > 0) ? 1u : 0u);
+            const bool fresh = SPLIT && p.oacc_T > 0 ? (s % p.oacc_T == 0) : (s == 0);
+            mma_ts(dcol, tmem + kTmemP + kk * 8, bd, idO, (!fresh || kk > 0) ? 1u : 0u);
             if (SPLIT) mma_ts(dcol, tmem + kTmemP + 64 + kk * 8, bd, idO, 1u);
           }
           for (int u = 0; u < run; ++u) tc_commit(&empty[st + u]);
@@ -698,6 +710,12 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     bool ok = true;
     Tracer str = tracer(2);
     if (threadIdx.x != 128) str.buf = nullptr;
+    // float32 inputs: this row's fp32 accumulator of the flushed O segments
+    const bool oseg = SPLIT && p.oacc_T > 0;
+    float* accrow = oseg ? reinterpret_cast<float*>(tail + p.oacc_off) + (size_t)(wq * 32 + lane) * (p.Ocols + 1)
+                         : nullptr;
+    if (oseg)
+      for (int c = 0; c <= p.Ocols; ++c) accrow[c] = 0.f;
     for (int s = 0; s < nkt; ++s) {
       const int kt = tiles[s];
       const int kb = s & 1;
@@ -848,7 +866,18 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
       }
       str.ev(25);
-      if (__any_sync(0xffffffffu, resc)) {
+      if (oseg && s > 0 && s % p.oacc_T == 0) {
+        // close the tensor-memory segment: O joins the row's accumulator (both
+        // rescaled to the current maximum) and P.V(s) starts a fresh one
+        const float f = resc ? alpha : 1.f;
+        for (int c = 0; c < p.Ocols; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) accrow[c + e] = (accrow[c + e] + __uint_as_float(o[e])) * f;
+        }
+      } else if (__any_sync(0xffffffffu, resc)) {
         const float f = resc ? alpha : 1.f;
         for (int c = 0; c < p.Ocols; c += 32) {
           uint32_t o[32];
@@ -858,6 +887,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
           tmem_st32(trow + (uint32_t)(p.tmemO + c), o);
         }
+        if (oseg)
+          for (int c = 0; c < p.Ocols; ++c) accrow[c] *= f;
       }
       tmem_st32(trow + kTmemP, pk[0]);
       tmem_st32(trow + kTmemP + 32, pk[1]);
@@ -929,6 +960,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tmem_ld32(tmem + ((uint32_t)((warp - 4) * 32) << 16) + (uint32_t)(p.tmemO + (p.ones_col & ~31)), o);
         tmem_ld_wait();
         lt = __uint_as_float(o[p.ones_col & 31]);
+        if (p.oacc_T > 0)
+          lt += reinterpret_cast<float*>(tail + p.oacc_off)[(size_t)((warp - 4) * 32 + lane) * (p.Ocols + 1) + p.ones_col];
       }
       rowlsum[(warp - 4) * 32 + lane] = lt;
     }
@@ -963,7 +996,8 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           tmem_ld32(trow + (uint32_t)(p.tmemO + c), o);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orow[c + e] = __uint_as_float(o[e]) * inv_o;
+          for (int e = 0; e < 32; ++e)
+            orow[c + e] = (SPLIT && p.oacc_T > 0 ? orow[c + e] + __uint_as_float(o[e]) : __uint_as_float(o[e])) * inv_o;
         }
       }
       ttr.ev(45);

@@ -39,6 +39,7 @@ constexpr int kVbufMinTiles = 8;  // key tiles from which the value-buffer mode 
 constexpr int kMaxPts = 64;      // points per head handled by the prologue scratch
 constexpr int kMaxRCz = 1024;    // R*Cz handled by the prologue scratch
 constexpr int kMaxTiles = 1024;  // key tiles per sample (N <= 131072)
+constexpr int kOaccTiles = 4;    // float32 inputs: key tiles per tensor-memory segment of O
 constexpr int kMaxPSimt = 16;    // points per head of the fp32 (exact distance) mode
 constexpr int kLiftRes = 8;      // most residues per prologue lift CTA (divides the 32-residue group)
 constexpr int kWpTiles = 4;      // 32x32 output-weight tiles per weight-preparation CTA
@@ -93,6 +94,8 @@ struct Plan {
   int Kq, nQc;        // Qhat row width and chunks
   int VHc, VHp, nVH;  // value head-part columns, padded, chunks
   int ones_col;       // float32 inputs: value column holding 1 (the P.V product's own sum of P), or -1
+  int oacc_T;         // float32 inputs: key tiles per tensor-memory segment of O (0 = one segment)
+  int oacc_off;       // tail offset of the per-row fp32 accumulator [128][Ocols + 1] (oacc_T > 0)
   int ZVc, nZV;       // pair columns used by the value product, chunks
   int Ocols;          // VHp + nZV * 64: fp32 accumulator columns per row
   int Pcols;          // TMEM columns holding P (64, or 128 for hi+lo)
@@ -191,8 +194,23 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   if (p.tmemO + p.Ocols > 512) { *why = "lifted value width exceeds the 512 tensor-memory columns"; return 2; }
   // core shared memory: resident Qhat + ring + barriers/buffers (+1 KB alignment slack)
   const size_t kp_bytes = p.geo_simt ? (size_t)2 * kTile * 3 * P * 4 : 0;
-  const size_t fixed = 1024 + 5120 + 2 * kMaxTiles + kp_bytes;   // slack + tail (see core.cu)
+  size_t fixed = 1024 + 5120 + 2 * kMaxTiles + kp_bytes;   // slack + tail (see core.cu)
   const size_t limit = 232448;  // 227 KB opt-in maximum per block on sm_100
+  // float32 inputs: the tensor cores accumulate O for kOaccTiles key tiles at a
+  // time, then the softmax warps add it into a per-row fp32 accumulator (round
+  // to nearest) in the tail, so no fp32 sum in tensor memory spans more than
+  // 16 x kOaccTiles key slices (its rounding drifts with the number of terms)
+  p.oacc_T = 0;
+  p.oacc_off = 0;
+  if (f32) {
+    const size_t oacc_bytes = (size_t)kTile * (p.Ocols + 1) * 4;
+    const size_t need = limit - (fixed + oacc_bytes) - (size_t)p.nQc * 16384;
+    if (fixed + oacc_bytes + (size_t)p.nQc * 16384 < limit && need / 16384 >= 3) {
+      p.oacc_T = kOaccTiles;
+      p.oacc_off = (int)(5120 + 2 * kMaxTiles + kp_bytes);
+      fixed += oacc_bytes;
+    }
+  }
   p.nVB = p.nVH + p.nZV;
   p.vbuf = 0;
   p.nQres = p.nQc;
@@ -214,7 +232,7 @@ static inline int make_plan(Plan& p, int B, int N, int H, int D, int Dv, int P, 
   const int nchunks = p.nQres + (p.vbuf ? p.nVB : 0) + nst;   // Qhat, value buffer, ring
   p.core_smem = fixed + (size_t)nchunks * 16384;
   if (p.core_smem < 120 * 1024) p.core_smem = 120 * 1024;   // one CTA per SM (TMEM is taken whole)
-  if ((size_t)kTile * (p.Ocols + 1) * 4 > (size_t)nchunks * 16384) {
+  if (p.oacc_T == 0 && (size_t)kTile * (p.Ocols + 1) * 4 > (size_t)nchunks * 16384) {
     *why = "value width too large for the epilogue staging"; return 2;
   }
   // prologue lift kernel: Wb^T, zero-padded z1 / q / k / v / point rows

@@ -49,10 +49,11 @@ def test_workload0_tiny_f32(handles):
 
 
 def test_workload0_float32_long_chain(handles):
-    """The float32 path on a long chain (N = 2048: 16 key tiles per query tile,
-    the exact point term over every key group, the aggregates normalised by
-    the tensor cores' own sum of P), on sampled rows."""
-    n = 2048
+    """The float32 path on a long chain (N = 4096: 32 key tiles per query tile,
+    the exact point term over every key group, O accumulated by the tensor
+    cores in segments of a few key tiles and added in fp32 on the CUDA cores,
+    normalised by its own sum of P), on sampled rows."""
+    n = 4096
     inp = workloads.make_inputs(workloads.workload(0).with_(N=n))
     rng = np.random.default_rng(40)
     rows = np.unique(np.concatenate([[0, 127, 128, n - 1], rng.choice(n, 60, replace=False)]))
