@@ -254,10 +254,11 @@ struct EpiLayout {
   uint32_t z1_row_bytes, z1_stride, o_off;
 };
 
+template <bool SPLIT>
 __device__ __forceinline__ EpiLayout epi_layout(const Plan& p, const void* z1) {
   EpiLayout e;
   const uint32_t ring_end = (uint32_t)(p.nQres + (p.vbuf ? p.nVB : 0) + p.nst) * kChunkBytes;
-  if (p.oacc_T > 0) {
+  if (SPLIT && p.oacc_T > 0) {
     // float32 inputs with O in segments: the rows are staged in place in the
     // fp32 accumulator (the tail), all columns, and z1 may use the Qhat region
     e.fast_pair = false;
@@ -614,8 +615,9 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint64_t bd = desc_mnmajor_sw128(b0 + kk * 2048, kChunkBytes);
-            const bool fresh = SPLIT && p.oacc_T > 0 ? (s % p.oacc_T == 0) : (s == 0);
-            mma_ts(dcol, tmem + kTmemP + kk * 8, bd, idO, (!fresh || kk > 0) ? 1u : 0u);
+            uint32_t acc0 = (s > 0 || kk > 0) ? 1u : 0u;
+            if (SPLIT && p.oacc_T > 0) acc0 = (s % p.oacc_T != 0 || kk > 0) ? 1u : 0u;
+            mma_ts(dcol, tmem + kTmemP + kk * 8, bd, idO, acc0);
             if (SPLIT) mma_ts(dcol, tmem + kTmemP + 64 + kk * 8, bd, idO, 1u);
           }
           for (int u = 0; u < run; ++u) tc_commit(&empty[st + u]);
@@ -911,7 +913,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       for (int e = 0; e < 9; ++e) rowR[e] = ld_any(a.rot, bi * 9 + e, p.in_f32);
 #pragma unroll
       for (int e = 0; e < 3; ++e) rowT[e] = ld_any(a.trans, bi * 3 + e, p.in_f32);
-      const EpiLayout el = epi_layout(p, a.z1);
+      const EpiLayout el = epi_layout<SPLIT>(p, a.z1);
       if (el.z1_smem && i < N) {
         const uint8_t* src = static_cast<const uint8_t*>(a.z1) + bi * el.z1_row_bytes;
         uint8_t* dst = smem + (size_t)(wq * 32 + lane) * el.z1_stride;
@@ -939,7 +941,7 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   ttr.ev(42);
-  const EpiLayout el = epi_layout(p, a.z1);
+  const EpiLayout el = epi_layout<SPLIT>(p, a.z1);
   const bool fast_pair = el.fast_pair;
   // per-row state for the warps that did not run the softmax (the key-term
   // buffer is free now); the z1 copies of the softmax threads complete first
