@@ -778,13 +778,38 @@ fipa_core_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 #pragma unroll
           for (int e = 0; e < 32; ++e) d2[e] = 0.f;
           const float* kt0 = kpb + t * 32 * P3;
-          for (int x = 0; x < P3; ++x) {
-            const int c = x % 3;
-            const float ax = aq[x] + (c == 0 ? dd[0] : (c == 1 ? dd[1] : dd[2]));
+          if ((P3 & 3) == 0) {
+            // four coordinates of a key per 16-byte load (rows of 3P floats stay
+            // 16-byte aligned), added in the same order
+            for (int x = 0; x < P3; x += 4) {
+              float ax[4];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float d = ax - kt0[e * P3 + x];
-              d2[e] = fmaf(d, d, d2[e]);
+              for (int u = 0; u < 4; ++u) {
+                const int c = (x + u) % 3;
+                ax[u] = aq[x + u] + (c == 0 ? dd[0] : (c == 1 ? dd[1] : dd[2]));
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float4 kv = *reinterpret_cast<const float4*>(kt0 + e * P3 + x);
+                float d = ax[0] - kv.x;
+                d2[e] = fmaf(d, d, d2[e]);
+                d = ax[1] - kv.y;
+                d2[e] = fmaf(d, d, d2[e]);
+                d = ax[2] - kv.z;
+                d2[e] = fmaf(d, d, d2[e]);
+                d = ax[3] - kv.w;
+                d2[e] = fmaf(d, d, d2[e]);
+              }
+            }
+          } else {
+            for (int x = 0; x < P3; ++x) {
+              const int c = x % 3;
+              const float ax = aq[x] + (c == 0 ? dd[0] : (c == 1 ? dd[1] : dd[2]));
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float d = ax - kt0[e * P3 + x];
+                d2[e] = fmaf(d, d, d2[e]);
+              }
             }
           }
 #pragma unroll
